@@ -1,0 +1,238 @@
+/*
+ * fathom.h -- C ABI of the Fathom top-k key scan on NVIDIA B200 (sm_100a).
+ *
+ * Fathom ("Fathom: Per-Query Read Depth for Sparse Decoding over Offloaded
+ * KV Caches", arXiv 2609.17652) scores all n cached keys of a KV head for
+ * its G query heads by reading only a query-chosen prefix of each key
+ * channel's 4-bit code, then keeps the top k keys per query head.  The
+ * passages cited below are sections of the yeyulingfeng.com article on the
+ * paper; "方法一" is the bit-plane store, "方法二" the per-group reverse
+ * water-filling, "先算一笔字节账" the byte accounting.
+ *
+ * Conventions for every entry point
+ *   - Memory is owned by the caller.  The library never allocates, never
+ *     frees and keeps no state between calls (except the per-thread last
+ *     CUDA error code).  Pointers marked DEVICE must be readable (or
+ *     writable) by the current CUDA device: device memory, managed memory,
+ *     or, where stated, page-locked host memory mapped into the device's
+ *     address space.  Pointers marked HOST are ordinary host memory.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) on the current device.  Outputs are valid
+ *     once the stream reaches the call.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing and returns a negative status.
+ *   - A "group" is one KV head of one layer (its G query heads share one
+ *     plan, so each key byte is read once, 方法二 last paragraph).  Arrays
+ *     indexed [H] run over the groups of one call.
+ *   - Layout names list dimensions outermost first; all arrays are dense
+ *     row-major unless a stride argument says otherwise.
+ *   - Limits: 32 <= D <= 256 with D % 32 == 0; 1 <= G <= 8; 1 <= k <= 4096
+ *     and G*k <= 16384 for top-k; n < 2^31.
+ */
+#ifndef FATHOM_H
+#define FATHOM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* fathom_stream_t; /* same type as cudaStream_t */
+
+/* Status codes. */
+#define FATHOM_OK 0
+#define FATHOM_ERR_INVALID_ARG (-1) /* null/unreadable pointer, size or range error */
+#define FATHOM_ERR_UNSUPPORTED (-2) /* D, G, k or alignment outside the limits above */
+#define FATHOM_ERR_CUDA (-3)        /* a CUDA call failed; see fathom_last_cuda_error() */
+#define FATHOM_ERR_WORKSPACE (-4)   /* caller buffer smaller than the *_bytes() query */
+#define FATHOM_ERR_TIMEOUT (-5)     /* reserved: a bounded device wait gave up */
+#define FATHOM_ERR_OVERFLOW (-6)    /* candidate pass could not prove its top-k exact */
+
+/* Key element types for fathom_pack. */
+#define FATHOM_KEYS_F32 0
+#define FATHOM_KEYS_BF16 1
+
+/* Output modes of fathom_scan. */
+#define FATHOM_SCAN_DENSE 0
+#define FATHOM_SCAN_CANDIDATE 1
+
+/* Library version as 10000*major + 100*minor + patch. */
+int fathom_version(void);
+
+/* Static, human-readable text for a status code. */
+const char* fathom_status_string(int status);
+
+/* The cudaError_t value behind the calling thread's last FATHOM_ERR_CUDA
+ * (0 if none). */
+int fathom_last_cuda_error(void);
+
+/* Words per plane row for n tokens: ceil(n/64) rounded up to a multiple of
+ * 16, i.e. 128-byte rows.  Any nb_stride >= ceil(n/64) that is even is
+ * accepted; this value is the recommended one. */
+int64_t fathom_nb_stride(int64_t n);
+
+/*
+ * fathom_pack -- build the bit-plane index of H groups (方法一).
+ *
+ * For group h, channel j and 64-token block b (tokens 64b .. 64b+63 that
+ * are < n):
+ *   m = max |k| over the block's tokens, s = m rounded to fp16 (nearest,
+ *   ties to even), and each key gets the 4-bit code
+ *   c = clamp(floor(8 k / s) + 8, 0, 15)    (c = 8 when s is 0 or infinite),
+ * i.e. 16 uniform cells of width s/8 over [-s, s]; code 8 is the cell
+ * [0, s/8) and the top bit of c is the sign (1 for k >= 0).  Plane p
+ * (p = 0 is the top bit, read first) of channel j holds bit (3-p) of the
+ * 64 codes of block b in one 64-bit word, token 64b+i at bit i:
+ *   planes[((h*D + j)*4 + p)*nb_stride + b],
+ * so each plane row is contiguous along the sequence.  Bits of tokens >= n
+ * are 0.  Storage: 4 x 8 B + 2 B per channel per 64 tokens = 68 B per token
+ * per KV head at D = 128.
+ *
+ *   keys        DEVICE, key_dtype elements; token i of group h, channel j at
+ *               keys[h*key_stride_h + i*key_stride_tok + j] (element units;
+ *               channels contiguous).  Values should be finite with
+ *               |k| < 65520 (fp16 range of the scale).
+ *   key_dtype   FATHOM_KEYS_F32 or FATHOM_KEYS_BF16.
+ *   H, n, D     groups, tokens, channels.  H == 0 or n == 0 is a no-op.
+ *   planes      DEVICE out, uint64 [H][D][4][nb_stride], 8-byte aligned.
+ *   scales      DEVICE out, fp16 bit patterns [H][D][nb_stride].
+ *   nb_stride   words per plane row, >= ceil(n/64) and even.
+ * Words/scales at block indices >= ceil(n/64) are not written.
+ */
+int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
+                int64_t key_stride_h, int64_t key_stride_tok,
+                uint64_t* planes, uint16_t* scales, int64_t nb_stride,
+                fathom_stream_t stream);
+
+/*
+ * fathom_plan -- per-group reverse water-filling (方法二).
+ *
+ * Channel importance, in single precision with round-to-nearest and in this
+ * exact order (no fused multiply-add):
+ *   w_j = sigma2_j * ((((q_{0,j}^2 + q_{1,j}^2) + q_{2,j}^2) + ...) + q_{G-1,j}^2).
+ * Reading t planes leaves error variance proportional to 4^-t, so the
+ * (t+1)-th plane of channel j is worth the item w_j * 4^-t (t = 0..3).
+ * The water level theta* is the smallest theta >= 0 for which
+ *   sum_j t_j(theta) <= B,  t_j(theta) = #{t in 0..3 : w_j 4^-t > theta},
+ * i.e. the (B+1)-th largest positive item, or 0 when at most B items are
+ * positive; depth_j = t_j(theta*).  Ties at theta* are all left unread, so
+ * sum_j depth_j can be below B.  Items are compared exactly.  The search is
+ * a bisection on an integer key that is monotone in log theta and ends
+ * exactly (at most 32 halvings).
+ *
+ *   sigma2       DEVICE, fp32 [H][D], per-channel key variance (calibration).
+ *   q            DEVICE, fp32 [H][G][D], the group's query heads.
+ *   budget_bits  DEVICE, int32 [H], plane bits per token per group (B); or
+ *                NULL to use budget_flat for every group.  Values are
+ *                clamped to [0, 4D].
+ *   budget_flat  used when budget_bits is NULL; must be in [0, 4D].
+ *   depth        DEVICE out, uint8 [H][D], t_j in 0..4.
+ *   active       DEVICE out, uint16 [H][D]: the channels with t_j > 0 in
+ *                ascending j, entry = j | (t_j << 8); entries past n_active
+ *                are 0.
+ *   n_active     DEVICE out, int32 [H].
+ *   theta        DEVICE out (may be NULL), fp32 [H]: theta* rounded to fp32
+ *                (informational; depths are decided exactly).
+ */
+int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D,
+                const int32_t* budget_bits, int32_t budget_flat,
+                uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
+                fathom_stream_t stream);
+
+/*
+ * fathom_plan_fixed -- the fixed-depth comparator plan: the r channels with
+ * the largest a_j = |q_{0,j}| + |q_{1,j}| + ... + |q_{G-1,j}| (single
+ * precision, that order; ties to the lower j) at depth 4, the others at 0.
+ * With r = 32 this is the 136-bit scan of the byte accounting
+ * (先算一笔字节账, third bullet: 32 coordinates x 4 bits + a block scale).
+ * The group's heads share the channel set so the K bytes are read once.
+ * Outputs as fathom_plan.  0 <= r <= D.
+ */
+int fathom_plan_fixed(const float* q, int64_t H, int G, int D, int r,
+                      uint8_t* depth, uint16_t* active, int32_t* n_active,
+                      fathom_stream_t stream);
+
+/*
+ * fathom_scan_cand_bytes -- size of the candidate buffer fathom_scan needs
+ * in FATHOM_SCAN_CANDIDATE mode for these sizes (HOST call, no GPU work).
+ */
+size_t fathom_scan_cand_bytes(int64_t H, int G, int64_t n, int k);
+
+/*
+ * fathom_scan -- variable-depth scores (方法一 prefix reads, 方法二 plan).
+ *
+ * For group h, query head g and token i < n:
+ *   score_{g,i} = sum_{(j,t) in active[h]} q_{g,j} * khat_{i,j},
+ *   khat = s_{b,j} * (2 c_t - 2^t + 1) / 2^t,   c_t = the first t planes'
+ * bits of the key's code (the t-bit mid-rise quantiser on [-s, s]), b = i/64.
+ * Only the first t plane rows of each active channel and its scale row are
+ * read; every plane word is read once for all G heads.  Arithmetic is fp32
+ * (coefficients q * s * 2^-t rounded once, one fused multiply-add per
+ * term); the result is within 1e-5 * sum_j |q_{g,j} khat_{i,j}| of exact
+ * for D <= 128.  No 1/sqrt(D) factor is applied (it does not change ranks).
+ *
+ *   planes, scales  DEVICE (or mapped page-locked host memory), as written
+ *                   by fathom_pack with the same nb_stride.  planes must be
+ *                   16-byte aligned and nb_stride even.
+ *   active, n_active  DEVICE, from fathom_plan / fathom_plan_fixed.
+ *   q               DEVICE, fp32 [H][G][D].
+ *   mode            FATHOM_SCAN_DENSE: write scores.
+ *                   FATHOM_SCAN_CANDIDATE: write into cand only the keys
+ *                   whose score reaches a per-head threshold tau taken
+ *                   from a 1-in-S tile sample of the same scores (S chosen
+ *                   from n and k; tau = -inf when n is small), so that
+ *                   fathom_topk can select from them.  The threshold is a
+ *                   filter only: fathom_topk checks that at least k keys
+ *                   passed and none were dropped, which proves the top-k
+ *                   exact, and flags the group otherwise.
+ *   scores          DEVICE out, fp32 [H][G][n] (DENSE; ignored otherwise).
+ *   cand, cand_bytes  DEVICE scratch/out of at least
+ *                   fathom_scan_cand_bytes(H, G, n, k) bytes (CANDIDATE;
+ *                   ignored in DENSE mode), 16-byte aligned.
+ *   k               winners per query head that will be asked of
+ *                   fathom_topk (sizes the candidate pass).
+ */
+int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D,
+                int64_t n, int64_t nb_stride, const uint16_t* active,
+                const int32_t* n_active, const float* q, int G, int mode,
+                float* scores, void* cand, size_t cand_bytes, int k,
+                fathom_stream_t stream);
+
+/*
+ * fathom_topk_workspace_bytes -- scratch fathom_topk needs (HOST call).
+ */
+size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k);
+
+/*
+ * fathom_topk -- per query head, the k keys with the largest scores, ties
+ * broken towards the lower token index, listed by (score descending, index
+ * ascending); then per group the ascending, de-duplicated union of its G
+ * winner lists (at most G*k keys; 先算一笔字节账, top-k bullet).
+ *
+ * Scores are ordered as fp32 values (-0 equals +0).  Exactly one of
+ * scores / cand is non-NULL:
+ *   scores     DEVICE, fp32 [H][G][n] from a DENSE scan.
+ *   cand       DEVICE, the candidate buffer of a CANDIDATE scan with the
+ *              same H, G, n, k.
+ *   idx        DEVICE out, int32 [H][G][k].
+ *   union_idx  DEVICE out, int32 [H][G*k], ascending, -1 padded.
+ *   union_count DEVICE out, int32 [H]: size of each union, or
+ *              FATHOM_ERR_OVERFLOW for a group whose candidate pass kept
+ *              fewer than k or more than its capacity of keys; such a
+ *              group's idx and union_idx are unspecified and the caller
+ *              reruns it with a DENSE scan.
+ *   workspace, ws_bytes  DEVICE scratch of fathom_topk_workspace_bytes()
+ *              bytes (may be NULL when that is 0).
+ */
+int fathom_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k,
+                int32_t* idx, int32_t* union_idx, int32_t* union_count,
+                void* workspace, size_t ws_bytes, fathom_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FATHOM_H */

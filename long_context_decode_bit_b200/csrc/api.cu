@@ -1,0 +1,223 @@
+// extern "C" entry points of libfathom.so (declared in include/fathom.h):
+// argument validation on the host, then the launches.  No allocation, no
+// state beyond the per-thread last CUDA error.
+#include "common.cuh"
+
+namespace fathom {
+
+int launch_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t stride_h,
+                int64_t stride_tok, uint64_t* planes, uint16_t* scales, int64_t nb_stride, cudaStream_t stream);
+int launch_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,
+                int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
+                cudaStream_t stream);
+int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, uint8_t* depth, uint16_t* active,
+                      int32_t* n_active, cudaStream_t stream);
+int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
+                const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
+                void* cand, int k, cudaStream_t stream);
+int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
+                int32_t* union_idx, int32_t* union_count, cudaStream_t stream);
+
+static thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return FATHOM_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return FATHOM_ERR_CUDA;
+}
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// A pointer the current device can dereference: device or managed memory,
+// or page-locked host memory mapped into the device's address space.
+int check_device_ptr(const void* p)
+{
+    if (!p) return FATHOM_ERR_INVALID_ARG;
+    cudaPointerAttributes attr;
+    const cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return FATHOM_ERR_INVALID_ARG;
+    }
+    switch (attr.type) {
+        case cudaMemoryTypeDevice:
+        case cudaMemoryTypeManaged:
+            return FATHOM_OK;
+        case cudaMemoryTypeHost:
+            return attr.devicePointer == p ? FATHOM_OK : FATHOM_ERR_INVALID_ARG;
+        default:
+            return FATHOM_ERR_INVALID_ARG;
+    }
+}
+
+bool dims_ok(int D, int G) { return D >= 32 && D <= kMaxD && D % 32 == 0 && G >= 1 && G <= kMaxG; }
+
+}  // namespace
+}  // namespace fathom
+
+using namespace fathom;
+
+#define FATHOM_TRY(expr)                 \
+    do {                                 \
+        const int _st = (expr);          \
+        if (_st != FATHOM_OK) return _st; \
+    } while (0)
+
+extern "C" {
+
+int fathom_version(void) { return 10000; }
+
+const char* fathom_status_string(int status)
+{
+    switch (status) {
+        case FATHOM_OK: return "ok";
+        case FATHOM_ERR_INVALID_ARG: return "invalid argument";
+        case FATHOM_ERR_UNSUPPORTED: return "unsupported size or alignment";
+        case FATHOM_ERR_CUDA: return "CUDA error";
+        case FATHOM_ERR_WORKSPACE: return "buffer too small";
+        case FATHOM_ERR_TIMEOUT: return "device wait timed out";
+        case FATHOM_ERR_OVERFLOW: return "candidate pass could not prove the top-k exact";
+        default: return "unknown status";
+    }
+}
+
+int fathom_last_cuda_error(void) { return g_last_cuda_error; }
+
+int64_t fathom_nb_stride(int64_t n)
+{
+    if (n <= 0) return 0;
+    return ceil_div(ceil_div(n, kBlockTokens), 16) * 16;
+}
+
+int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t key_stride_h,
+                int64_t key_stride_tok, uint64_t* planes, uint16_t* scales, int64_t nb_stride,
+                fathom_stream_t stream)
+{
+    if (H < 0 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
+    if (key_dtype != FATHOM_KEYS_F32 && key_dtype != FATHOM_KEYS_BF16) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
+    if (H == 0 || n == 0) return FATHOM_OK;
+    const int64_t nb = ceil_div(n, kBlockTokens);
+    if (nb_stride < nb || (nb_stride & 1)) return FATHOM_ERR_INVALID_ARG;
+    if (key_stride_tok < D || (H > 1 && key_stride_h < n * key_stride_tok)) return FATHOM_ERR_INVALID_ARG;
+    if (H > 65535 / (D / 32)) return FATHOM_ERR_UNSUPPORTED;
+    if (!aligned(planes, 8) || !aligned(scales, 2) || !aligned(keys, key_dtype == FATHOM_KEYS_F32 ? 4 : 2))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(keys));
+    FATHOM_TRY(check_device_ptr(planes));
+    FATHOM_TRY(check_device_ptr(scales));
+    return launch_pack(keys, key_dtype, H, n, D, key_stride_h, key_stride_tok, planes, scales, nb_stride,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,
+                int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
+                fathom_stream_t stream)
+{
+    if (H < 0 || H > 0x7FFFFFFF) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
+    if (!budget_bits && (budget_flat < 0 || budget_flat > 4 * D)) return FATHOM_ERR_INVALID_ARG;
+    if (H == 0) return FATHOM_OK;
+    if (!aligned(sigma2, 4) || !aligned(q, 4) || !aligned(active, 2) || !aligned(n_active, 4) ||
+        (budget_bits && !aligned(budget_bits, 4)) || (theta && !aligned(theta, 4)))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(sigma2));
+    FATHOM_TRY(check_device_ptr(q));
+    FATHOM_TRY(check_device_ptr(depth));
+    FATHOM_TRY(check_device_ptr(active));
+    FATHOM_TRY(check_device_ptr(n_active));
+    if (budget_bits) FATHOM_TRY(check_device_ptr(budget_bits));
+    if (theta) FATHOM_TRY(check_device_ptr(theta));
+    return launch_plan(sigma2, q, H, G, D, budget_bits, budget_flat, depth, active, n_active, theta,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fathom_plan_fixed(const float* q, int64_t H, int G, int D, int r, uint8_t* depth, uint16_t* active,
+                      int32_t* n_active, fathom_stream_t stream)
+{
+    if (H < 0 || H > 0x7FFFFFFF) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
+    if (r < 0 || r > D) return FATHOM_ERR_INVALID_ARG;
+    if (H == 0) return FATHOM_OK;
+    if (!aligned(q, 4) || !aligned(active, 2) || !aligned(n_active, 4)) return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(q));
+    FATHOM_TRY(check_device_ptr(depth));
+    FATHOM_TRY(check_device_ptr(active));
+    FATHOM_TRY(check_device_ptr(n_active));
+    return launch_plan_fixed(q, H, G, D, r, depth, active, n_active, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fathom_scan_cand_bytes(int64_t H, int G, int64_t n, int k)
+{
+    if (H <= 0 || G < 1 || G > kMaxG || n <= 0 || k < 1 || k > n) return 0;
+    return cand_layout(H, G, n, k).total;
+}
+
+int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
+                const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
+                void* cand, size_t cand_bytes, int k, fathom_stream_t stream)
+{
+    if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
+    if (mode != FATHOM_SCAN_DENSE && mode != FATHOM_SCAN_CANDIDATE) return FATHOM_ERR_INVALID_ARG;
+    if (H == 0 || n == 0) return FATHOM_OK;
+    const int64_t nb = ceil_div(n, kBlockTokens);
+    if (nb_stride < nb) return FATHOM_ERR_INVALID_ARG;
+    if ((nb_stride & 1) || !aligned(planes, 16) || !aligned(scales, 2) || !aligned(active, 2) ||
+        !aligned(n_active, 4) || !aligned(q, 4))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(planes));
+    FATHOM_TRY(check_device_ptr(scales));
+    FATHOM_TRY(check_device_ptr(active));
+    FATHOM_TRY(check_device_ptr(n_active));
+    FATHOM_TRY(check_device_ptr(q));
+    if (mode == FATHOM_SCAN_DENSE) {
+        if (!aligned(scores, 4)) return FATHOM_ERR_UNSUPPORTED;
+        FATHOM_TRY(check_device_ptr(scores));
+    } else {
+        if (k < 1 || k > n) return FATHOM_ERR_INVALID_ARG;
+        if (k > kMaxK) return FATHOM_ERR_UNSUPPORTED;
+        if (!aligned(cand, 16)) return FATHOM_ERR_UNSUPPORTED;
+        FATHOM_TRY(check_device_ptr(cand));
+        if (cand_bytes < cand_layout(H, G, n, k).total) return FATHOM_ERR_WORKSPACE;
+    }
+    return launch_scan(planes, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, k,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k)
+{
+    (void)H; (void)G; (void)n; (void)k;
+    return 0;
+}
+
+int fathom_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
+                int32_t* union_idx, int32_t* union_count, void* workspace, size_t ws_bytes,
+                fathom_stream_t stream)
+{
+    (void)workspace; (void)ws_bytes;
+    if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
+    if (G < 1 || G > kMaxG) return FATHOM_ERR_UNSUPPORTED;
+    if ((scores == nullptr) == (cand == nullptr)) return FATHOM_ERR_INVALID_ARG;
+    if (H == 0) return FATHOM_OK;
+    if (k < 1 || k > n) return FATHOM_ERR_INVALID_ARG;
+    if (k > kMaxK || static_cast<int64_t>(G) * k > kMaxUnion) return FATHOM_ERR_UNSUPPORTED;
+    if (!aligned(idx, 4) || !aligned(union_idx, 4) || !aligned(union_count, 4)) return FATHOM_ERR_UNSUPPORTED;
+    if (scores) {
+        if (!aligned(scores, 4)) return FATHOM_ERR_UNSUPPORTED;
+        FATHOM_TRY(check_device_ptr(scores));
+    } else {
+        if (!aligned(cand, 16)) return FATHOM_ERR_UNSUPPORTED;
+        FATHOM_TRY(check_device_ptr(cand));
+    }
+    FATHOM_TRY(check_device_ptr(idx));
+    FATHOM_TRY(check_device_ptr(union_idx));
+    FATHOM_TRY(check_device_ptr(union_count));
+    return launch_topk(scores, cand, H, G, n, k, idx, union_idx, union_count,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// Shared device helpers and launch plumbing for the Fathom kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "fathom.h"
+
+namespace fathom {
+
+constexpr int kBlockTokens = 64;   // tokens per scale block (one plane word)
+constexpr int kPlanes = 4;         // 4-bit codes
+constexpr int kMaxD = 256;
+constexpr int kMaxG = 8;
+constexpr int kMaxK = 4096;
+constexpr int kMaxUnion = 16384;
+
+// Record a CUDA error for fathom_last_cuda_error() and map it to a status.
+int cuda_status(cudaError_t e);
+
+// Launch-error check after a <<<>>> launch.
+inline int launch_status() { return cuda_status(cudaGetLastError()); }
+
+// ---------------------------------------------------------------------
+// Order-preserving map from fp32 to uint32: larger float -> larger key.
+// -0 is folded onto +0 so that the two compare equal, as fp32 values do.
+// ---------------------------------------------------------------------
+__device__ __forceinline__ uint32_t order_key(float f)
+{
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t k)
+{
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+    return __uint_as_float(u);
+}
+
+// ---------------------------------------------------------------------
+// Candidate buffer of a CANDIDATE scan.  Per (group, head): a header,
+// a sample-score area (only when a threshold is sampled) and `cap`
+// (index, score) entries.
+// ---------------------------------------------------------------------
+struct CandHeader {
+    int32_t count;   // keys that reached tau (may exceed cap: those were dropped)
+    float tau;       // threshold the main pass used
+    int32_t n_sample;
+    int32_t pad;
+};
+
+struct CandLayout {
+    int64_t heads;        // H * G
+    int64_t cap;          // entries per head
+    int64_t sample_tiles; // tiles in the sample (0: tau = -inf, no sample)
+    int64_t tile_stride;  // sample takes every tile_stride-th tile
+    int64_t n_sample;     // sample tokens per head (sample_tiles * tile tokens)
+    int64_t m_rank;       // tau = m_rank-th largest sample score
+    size_t off_hdr, off_sample, off_entries, total;
+};
+
+constexpr int kScanTileBlocks = 16;                       // 1024 tokens per scan tile
+constexpr int kScanTileTokens = kScanTileBlocks * kBlockTokens;
+
+CandLayout cand_layout(int64_t H, int G, int64_t n, int k);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace fathom

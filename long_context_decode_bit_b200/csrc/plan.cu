@@ -1,0 +1,166 @@
+// fathom_plan / fathom_plan_fixed: the per-group read plan.
+//
+// Reverse water-filling (Fathom, section "方法二"): the (t+1)-th plane of
+// channel j is worth the item w_j * 4^-t; the water level theta* is the
+// smallest theta whose item count above it fits the budget, and each
+// channel's depth is its number of items above theta*.  One CTA plans one
+// group, one thread per channel.  theta is searched by bisection over an
+// integer key that orders items exactly and grows like log2(theta): the
+// fp32 exponent and fraction of w, with the exponent extended below the
+// subnormal range and lowered by 2t for the factor 4^-t.
+#include "common.cuh"
+
+namespace fathom {
+
+namespace {
+
+// Exact, order-preserving key of the positive value w * 4^-t (w a positive
+// finite fp32).  key = (extended biased exponent) * 2^23 + fraction.
+__device__ __forceinline__ int32_t item_key(float w, int t)
+{
+    const uint32_t u = __float_as_uint(w);
+    int e = static_cast<int>((u >> 23) & 0xFF);
+    uint32_t f = u & 0x7FFFFFu;
+    if (e == 0) {                      // subnormal: normalise the fraction
+        const int msb = 31 - __clz(f);  // 0..22
+        e = msb - 22;                   // extended exponent, <= 0
+        f = (f << (23 - msb)) & 0x7FFFFFu;
+    }
+    return (e - 2 * t) * (1 << 23) + static_cast<int32_t>(f);
+}
+
+__device__ __forceinline__ float key_value(int32_t key)
+{
+    const int e = key >> 23;  // arithmetic shift: floor division
+    const uint32_t f = static_cast<uint32_t>(key) & 0x7FFFFFu;
+    if (e >= 1) return __uint_as_float(static_cast<uint32_t>(key));
+    return ldexpf(1.0f + static_cast<float>(f) * 0x1p-23f, e - 127);
+}
+
+// Compact (j, t) pairs with t > 0 into ascending-j active entries.
+__device__ __forceinline__ void write_active(int j, int t, int D, int64_t h, uint16_t* active,
+                                             int32_t* n_active, int* warp_cnt)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const unsigned bal = __ballot_sync(0xffffffffu, t > 0);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int base = 0, total = 0;
+    for (int w = 0; w < nwarps; ++w) {
+        if (w < warp) base += warp_cnt[w];
+        total += warp_cnt[w];
+    }
+    const int pos = base + __popc(bal & ((1u << lane) - 1u));
+    uint16_t* act = active + h * D;
+    if (t > 0) act[pos] = static_cast<uint16_t>(j | (t << 8));
+    if (j >= total) act[j] = 0;   // positions past n_active, exactly once each
+    if (j == 0) n_active[h] = total;
+}
+
+__global__ void plan_kernel(const float* __restrict__ sigma2, const float* __restrict__ q, int G, int D,
+                            const int32_t* __restrict__ budget_bits, int32_t budget_flat,
+                            uint8_t* __restrict__ depth, uint16_t* __restrict__ active,
+                            int32_t* __restrict__ n_active, float* __restrict__ theta)
+{
+    __shared__ int warp_cnt[kMaxD / 32];
+    __shared__ int red_min[kMaxD / 32], red_max[kMaxD / 32];
+    const int64_t h = blockIdx.x;
+    const int j = threadIdx.x;   // blockDim.x == D
+    const int lane = j & 31, warp = j >> 5, nwarps = D >> 5;
+
+    // Importance in the plan's fixed single-precision order (no FMA).
+    const float* qh = q + h * G * D + j;
+    float acc = __fmul_rn(qh[0], qh[0]);
+    for (int g = 1; g < G; ++g) acc = __fadd_rn(acc, __fmul_rn(qh[g * D], qh[g * D]));
+    const float w = __fmul_rn(sigma2[h * D + j], acc);
+    const bool pos = w > 0.0f;   // NaN and non-positive importance never read
+
+    int B = budget_bits ? budget_bits[h] : budget_flat;
+    B = min(max(B, 0), 4 * D);
+
+    int32_t k0 = 0, k3 = 0;
+    if (pos) { k0 = item_key(w, 0); k3 = item_key(w, 3); }
+    const int npos = __syncthreads_count(pos);
+
+    int32_t kstar;          // items with key > kstar are read
+    bool all_positive = false;
+    if (npos == 0 || 4 * npos <= B) {
+        all_positive = true;
+        kstar = 0;
+    } else {
+        // Range of item keys, for the bisection bounds.
+        int32_t mn = pos ? k3 : INT32_MAX, mx = pos ? k0 : INT32_MIN;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        if (lane == 0) { red_min[warp] = mn; red_max[warp] = mx; }
+        __syncthreads();
+        mn = INT32_MAX; mx = INT32_MIN;
+        for (int wi = 0; wi < nwarps; ++wi) { mn = min(mn, red_min[wi]); mx = max(mx, red_max[wi]); }
+        // Invariant: count(lo) > B >= count(hi); count(K) = #items with key > K.
+        int64_t lo = static_cast<int64_t>(mn) - 1, hi = mx;
+        int32_t kj[4] = {k0, pos ? item_key(w, 1) : 0, pos ? item_key(w, 2) : 0, k3};
+        while (hi - lo > 1) {
+            const int64_t mid = lo + ((hi - lo) >> 1);
+            int c = 0;
+            for (int r = 0; r < 4; ++r) c += __syncthreads_count(pos && kj[r] > mid);
+            if (c <= B) hi = mid; else lo = mid;
+        }
+        kstar = static_cast<int32_t>(hi);
+    }
+
+    int t = 0;
+    if (pos) {
+        if (all_positive) t = 4;
+        else
+            for (int r = 0; r < 4; ++r) t += item_key(w, r) > kstar;
+    }
+    depth[h * D + j] = static_cast<uint8_t>(t);
+    if (theta && j == 0) theta[h] = all_positive ? 0.0f : key_value(kstar);
+    write_active(j, t, D, h, active, n_active, warp_cnt);
+}
+
+__global__ void plan_fixed_kernel(const float* __restrict__ q, int G, int D, int r,
+                                  uint8_t* __restrict__ depth, uint16_t* __restrict__ active,
+                                  int32_t* __restrict__ n_active)
+{
+    __shared__ float a_s[kMaxD];
+    __shared__ int warp_cnt[kMaxD / 32];
+    const int64_t h = blockIdx.x;
+    const int j = threadIdx.x;
+    const float* qh = q + h * G * D + j;
+    float a = fabsf(qh[0]);
+    for (int g = 1; g < G; ++g) a = __fadd_rn(a, fabsf(qh[g * D]));
+    a_s[j] = a;
+    __syncthreads();
+    int rank = 0;
+    for (int i = 0; i < D; ++i) {
+        const float b = a_s[i];
+        rank += (b > a) || (b == a && i < j);
+    }
+    const int t = rank < r ? 4 : 0;
+    depth[h * D + j] = static_cast<uint8_t>(t);
+    write_active(j, t, D, h, active, n_active, warp_cnt);
+}
+
+}  // namespace
+
+int launch_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,
+                int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
+                cudaStream_t stream)
+{
+    plan_kernel<<<static_cast<unsigned>(H), D, 0, stream>>>(sigma2, q, G, D, budget_bits, budget_flat,
+                                                          depth, active, n_active, theta);
+    return launch_status();
+}
+
+int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, uint8_t* depth, uint16_t* active,
+                      int32_t* n_active, cudaStream_t stream)
+{
+    plan_fixed_kernel<<<static_cast<unsigned>(H), D, 0, stream>>>(q, G, D, r, depth, active, n_active);
+    return launch_status();
+}
+
+}  // namespace fathom

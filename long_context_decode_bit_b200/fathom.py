@@ -1,0 +1,256 @@
+"""ctypes binding of ``libfathom.so`` (C ABI in ``include/fathom.h``).
+
+Argument marshalling only: every step of the scan runs in the library's
+CUDA kernels.  torch tensors supply device memory and the current stream;
+outputs are allocated here with torch when the caller does not pass them.
+If the library is missing or cannot be loaded, every call raises -- there
+is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfathom.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_CUDA = -3
+ERR_WORKSPACE = -4
+ERR_TIMEOUT = -5
+ERR_OVERFLOW = -6
+
+KEYS_F32 = 0
+KEYS_BF16 = 1
+SCAN_DENSE = 0
+SCAN_CANDIDATE = 1
+
+# Every symbol include/fathom.h declares.
+EXPORTS = (
+    "fathom_version", "fathom_status_string", "fathom_last_cuda_error", "fathom_nb_stride",
+    "fathom_pack", "fathom_plan", "fathom_plan_fixed", "fathom_scan_cand_bytes", "fathom_scan",
+    "fathom_topk_workspace_bytes", "fathom_topk",
+)
+
+_lib = None
+
+
+class FathomError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = f"{what}: {_lib.fathom_status_string(status).decode() if _lib else status}"
+        if status == ERR_CUDA and _lib is not None:
+            msg += f" (cudaError {_lib.fathom_last_cuda_error()})"
+        super().__init__(msg)
+
+
+def load(path: str = LIB_PATH):
+    """Load the shared library (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} is missing: build it with `python -m long_context_decode_bit_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "fathom_version": (I, []),
+        "fathom_status_string": (ctypes.c_char_p, [I]),
+        "fathom_last_cuda_error": (I, []),
+        "fathom_nb_stride": (I64, [I64]),
+        "fathom_pack": (I, [P, I, I64, I64, I, I64, I64, P, P, I64, P]),
+        "fathom_plan": (I, [P, P, I64, I, I, P, ctypes.c_int32, P, P, P, P, P]),
+        "fathom_plan_fixed": (I, [P, I64, I, I, I, P, P, P, P]),
+        "fathom_scan_cand_bytes": (SZ, [I64, I, I64, I]),
+        "fathom_scan": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, SZ, I, P]),
+        "fathom_topk_workspace_bytes": (SZ, [I64, I, I64, I]),
+        "fathom_topk": (I, [P, P, I64, I, I64, I, P, P, P, P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def lib():
+    return load()
+
+
+def _check(st: int, what: str):
+    if st != OK:
+        raise FathomError(st, what)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def nb_stride(n: int) -> int:
+    return int(lib().fathom_nb_stride(int(n)))
+
+
+def scan_cand_bytes(H: int, G: int, n: int, k: int) -> int:
+    return int(lib().fathom_scan_cand_bytes(H, G, n, k))
+
+
+def topk_workspace_bytes(H: int, G: int, n: int, k: int) -> int:
+    return int(lib().fathom_topk_workspace_bytes(H, G, n, k))
+
+
+def pack(keys: torch.Tensor, nb_stride_words: int | None = None, planes=None, scales=None, stream=None):
+    """Bit-plane index of keys [H][n][D] (fp32 or bf16, channels contiguous).
+    Returns (planes uint64-as-int64 [H][D][4][nb_stride], scales int16 [H][D][nb_stride])."""
+    H, n, D = keys.shape
+    if keys.stride(2) != 1:
+        raise ValueError("keys must be contiguous along channels")
+    dt = {torch.float32: KEYS_F32, torch.bfloat16: KEYS_BF16}[keys.dtype]
+    nbs = nb_stride(n) if nb_stride_words is None else int(nb_stride_words)
+    dev = keys.device
+    if planes is None:
+        planes = torch.zeros((H, D, 4, nbs), dtype=torch.int64, device=dev)
+    if scales is None:
+        scales = torch.zeros((H, D, nbs), dtype=torch.int16, device=dev)
+    _check(lib().fathom_pack(_p(keys), dt, H, n, D, keys.stride(0), keys.stride(1), _p(planes), _p(scales),
+                             nbs, _stream(stream)), "fathom_pack")
+    return planes, scales
+
+
+def plan(sigma2: torch.Tensor, q: torch.Tensor, budget, out=None, stream=None):
+    """Reverse water-filling plan.  ``budget`` is an int (flat) or an int32
+    device tensor [H].  Returns (depth uint8 [H][D], active int16 [H][D],
+    n_active int32 [H], theta fp32 [H])."""
+    H, G, D = q.shape
+    dev = q.device
+    if out is None:
+        out = (torch.empty((H, D), dtype=torch.uint8, device=dev), torch.empty((H, D), dtype=torch.int16, device=dev),
+               torch.empty(H, dtype=torch.int32, device=dev), torch.empty(H, dtype=torch.float32, device=dev))
+    depth, active, n_active, theta = out
+    if isinstance(budget, torch.Tensor):
+        bptr, flat = _p(budget), 0
+    else:
+        bptr, flat = None, int(budget)
+    _check(lib().fathom_plan(_p(sigma2), _p(q), H, G, D, bptr, flat, _p(depth), _p(active), _p(n_active),
+                             _p(theta), _stream(stream)), "fathom_plan")
+    return depth, active, n_active, theta
+
+
+def plan_fixed(q: torch.Tensor, r: int, out=None, stream=None):
+    H, G, D = q.shape
+    dev = q.device
+    if out is None:
+        out = (torch.empty((H, D), dtype=torch.uint8, device=dev), torch.empty((H, D), dtype=torch.int16, device=dev),
+               torch.empty(H, dtype=torch.int32, device=dev))
+    depth, active, n_active = out
+    _check(lib().fathom_plan_fixed(_p(q), H, G, D, int(r), _p(depth), _p(active), _p(n_active), _stream(stream)),
+           "fathom_plan_fixed")
+    return depth, active, n_active
+
+
+def scan(planes, scales, n: int, active, n_active, q, mode: int = SCAN_DENSE, k: int = 0,
+         scores=None, cand=None, stream=None):
+    """Scores [H][G][n] (DENSE) or the candidate buffer (CANDIDATE)."""
+    H, G, D = q.shape
+    nbs = planes.shape[-1]
+    if mode == SCAN_DENSE:
+        if scores is None:
+            scores = torch.empty((H, G, n), dtype=torch.float32, device=q.device)
+        _check(lib().fathom_scan(_p(planes), _p(scales), H, D, n, nbs, _p(active), _p(n_active), _p(q), G,
+                                 SCAN_DENSE, _p(scores), None, 0, int(k), _stream(stream)), "fathom_scan")
+        return scores
+    nbytes = scan_cand_bytes(H, G, n, k)
+    if cand is None:
+        cand = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check(lib().fathom_scan(_p(planes), _p(scales), H, D, n, nbs, _p(active), _p(n_active), _p(q), G,
+                             SCAN_CANDIDATE, None, _p(cand), cand.numel() * cand.element_size(), int(k),
+                             _stream(stream)), "fathom_scan")
+    return cand
+
+
+def topk(H: int, G: int, n: int, k: int, scores=None, cand=None, out=None, workspace=None, stream=None):
+    """Per-head top-k and per-group union.  Returns (idx int32 [H][G][k],
+    union int32 [H][G*k], union_count int32 [H])."""
+    dev = (scores if scores is not None else cand).device
+    if out is None:
+        out = (torch.empty((H, G, k), dtype=torch.int32, device=dev),
+               torch.empty((H, G * k), dtype=torch.int32, device=dev),
+               torch.empty(H, dtype=torch.int32, device=dev))
+    idx, uni, cnt = out
+    ws_need = topk_workspace_bytes(H, G, n, k)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().fathom_topk(_p(scores), _p(cand), H, G, n, int(k), _p(idx), _p(uni), _p(cnt), _p(workspace),
+                             ws_bytes, _stream(stream)), "fathom_topk")
+    return idx, uni, cnt
+
+
+class Step:
+    """One decode step of the scan over a resident index: plan -> candidate
+    scan -> top-k + union, with the dense rerun for any group whose
+    candidate pass could not prove its top-k exact.  Buffers are allocated
+    once; ``run`` launches only library kernels."""
+
+    def __init__(self, planes, scales, n: int, sigma2, G: int, k: int, budget=48, fixed_r: int | None = None):
+        self.planes, self.scales, self.n, self.sigma2, self.k = planes, scales, n, sigma2, k
+        self.H, self.D = sigma2.shape
+        self.G = G
+        self.budget = budget
+        self.fixed_r = fixed_r
+        dev = sigma2.device
+        H, D = self.H, self.D
+        self.plan_out = (torch.empty((H, D), dtype=torch.uint8, device=dev),
+                         torch.empty((H, D), dtype=torch.int16, device=dev),
+                         torch.empty(H, dtype=torch.int32, device=dev),
+                         torch.empty(H, dtype=torch.float32, device=dev))
+        self.cand = torch.empty(scan_cand_bytes(H, G, n, k), dtype=torch.uint8, device=dev)
+        self.topk_out = (torch.empty((H, G, k), dtype=torch.int32, device=dev),
+                         torch.empty((H, G * k), dtype=torch.int32, device=dev),
+                         torch.empty(H, dtype=torch.int32, device=dev))
+        self.launches = 0
+
+    def run_plan(self, q):
+        if self.fixed_r is None:
+            plan(self.sigma2, q, self.budget, out=self.plan_out)
+        else:
+            plan_fixed(q, self.fixed_r, out=self.plan_out[:3])
+        return self.plan_out
+
+    def run_scan(self, q):
+        _, active, n_active, _ = self.plan_out
+        return scan(self.planes, self.scales, self.n, active, n_active, q, SCAN_CANDIDATE, self.k, cand=self.cand)
+
+    def run_topk(self):
+        return topk(self.H, self.G, self.n, self.k, cand=self.cand, out=self.topk_out)
+
+    def run(self, q, check_overflow: bool = True):
+        self.run_plan(q)
+        self.run_scan(q)
+        idx, uni, cnt = self.run_topk()
+        if check_overflow:
+            self.repair(q)
+        return idx, uni, cnt
+
+    def repair(self, q) -> int:
+        """Dense rerun of groups whose candidate pass overflowed (host check)."""
+        idx, uni, cnt = self.topk_out
+        bad = torch.nonzero(cnt < 0).flatten().tolist()
+        if not bad:
+            return 0
+        _, active, n_active, _ = self.plan_out
+        for h in bad:
+            sl = slice(h, h + 1)
+            sc = scan(self.planes[sl], self.scales[sl], self.n, active[sl], n_active[sl], q[sl], SCAN_DENSE)
+            topk(1, self.G, self.n, self.k, scores=sc, out=(idx[sl], uni[sl], cnt[sl]))
+        return len(bad)

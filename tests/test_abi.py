@@ -1,0 +1,81 @@
+"""The C-ABI library loads and exports every symbol include/fathom.h
+declares; host-only entry points and argument checks that return before
+any CUDA call behave as documented (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_decode_bit_b200 import build, fathom
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fathom.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return fathom.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fathom_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(fathom.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(fathom.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_host_only_entry_points(lib):
+    assert lib.fathom_version() == 10000
+    assert lib.fathom_status_string(0) == b"ok"
+    assert b"exact" in lib.fathom_status_string(-6)
+    assert lib.fathom_last_cuda_error() == 0
+    assert lib.fathom_nb_stride(1) == 16
+    assert lib.fathom_nb_stride(1024) == 16
+    assert lib.fathom_nb_stride(1025) == 32
+    assert lib.fathom_nb_stride(2 ** 20) == 16384
+    assert lib.fathom_topk_workspace_bytes(288, 4, 2 ** 20, 512) == 0
+    assert lib.fathom_scan_cand_bytes(0, 4, 100, 1) == 0
+    assert lib.fathom_scan_cand_bytes(1, 4, 100, 101) == 0   # k > n
+    small = lib.fathom_scan_cand_bytes(2, 4, 1000, 64)        # no sample: cap = n
+    assert small >= 2 * 4 * (16 + 1000 * 8)
+    big = lib.fathom_scan_cand_bytes(288, 4, 2 ** 20, 512)
+    # 1152 heads x (4096 entries of 8 B + 32768 sample scores of 4 B) + headers
+    assert big >= 1152 * (4096 * 8 + 32768 * 4)
+    assert big < 1152 * (4096 * 8 + 32768 * 4) + 1152 * 16 + 4096
+
+
+def test_rejections_before_any_cuda_call(lib):
+    n = None
+    # unsupported D and G, bad dtype, bad mode, bad budget: rejected on sizes alone
+    assert lib.fathom_pack(n, 0, 1, 64, 48, 64 * 48, 48, n, n, 16, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_pack(n, 7, 1, 64, 128, 64 * 128, 128, n, n, 16, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_pack(n, 0, 0, 64, 128, 0, 128, n, n, 16, n) == fathom.OK        # nothing to do
+    assert lib.fathom_plan(n, n, 4, 9, 128, n, 48, n, n, n, n, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_plan(n, n, 4, 4, 128, n, 513, n, n, n, n, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_plan(n, n, 4, 4, 128, n, -1, n, n, n, n, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_plan_fixed(n, 4, 4, 128, 129, n, n, n, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_scan(n, n, 1, 128, 100, 2, n, n, n, 4, 5, n, n, 0, 1, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_scan(n, n, 1, 100, 100, 2, n, n, n, 4, 0, n, n, 0, 1, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_topk(n, n, 1, 4, 100, 5, n, n, n, n, 0, n) == fathom.ERR_INVALID_ARG   # neither input
+    assert lib.fathom_topk(n, n, 1, 0, 100, 5, n, n, n, n, 0, n) == fathom.ERR_UNSUPPORTED   # G = 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = fathom._lib
+    fathom._lib = None
+    try:
+        with pytest.raises(FileNotFoundError):
+            fathom.load(str(tmp_path / "nope.so"))
+    finally:
+        fathom._lib = saved

@@ -1,0 +1,207 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.  Planes, scales and plans must be bit-exact; scores
+within 1e-5 of their L1 scale; top-k sets equal up to ties at the k-th
+score; top-k of the GPU's own scores identical to a full sort of them."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_decode_bit_b200 import inputs
+from _util import (assert_scores_close, assert_topk_sets_match, depth_to_active, keys_for_oracle,
+                   lexsort_topk, np_u16, np_u64)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def make(w, dev=DEV):
+    k = inputs.keys(w, 0, w.H, device=dev)
+    q = inputs.queries(w, 0, w.H, device=dev).float().contiguous()
+    s2 = inputs.calibration_sigma2(k, w.n_cal).contiguous()
+    return k, q, s2
+
+
+def oracle_pack(orc, k, nbs):
+    return orc.pack(keys_for_oracle(k), nb_stride=nbs)
+
+
+CASES = [
+    inputs.TINY,
+    dataclasses.replace(inputs.TINY, name="ragged", H=3, n=5037, seed=7),
+    dataclasses.replace(inputs.TINY, name="one-block", H=2, n=64, seed=8, n_cal=64),
+    dataclasses.replace(inputs.TINY, name="sub-block", H=2, n=37, seed=9, n_cal=37),
+    dataclasses.replace(inputs.LAYER_32K, name="qk-ragged", H=2, n=9000, seed=10),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_pack_bit_exact(fathom_gpu, orc, w):
+    k, _, _ = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    torch.cuda.synchronize()
+    p_ref, s_ref = oracle_pack(orc, k, planes.shape[-1])
+    assert np.array_equal(np_u64(planes), p_ref)
+    assert np.array_equal(np_u16(scales), s_ref)
+
+
+@pytest.mark.parametrize("D,G", [(32, 1), (64, 3), (256, 8)])
+def test_pack_plan_scan_other_shapes(fathom_gpu, orc, D, G):
+    w = dataclasses.replace(inputs.TINY, name=f"d{D}g{G}", H=2, n=3000, D=D, G=G, seed=11 + D)
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    depth, active, na, _ = fathom_gpu.plan(s2, q, min(4 * D, 3 * D // 2))
+    sc = fathom_gpu.scan(planes, scales, w.n, active, na, q)
+    torch.cuda.synchronize()
+    p_ref, s_ref = oracle_pack(orc, k, planes.shape[-1])
+    assert np.array_equal(np_u64(planes), p_ref) and np.array_equal(np_u16(scales), s_ref)
+    d_ref, a_ref, na_ref, _ = orc.plan(s2.cpu().numpy(), q.cpu().numpy(), min(4 * D, 3 * D // 2))
+    assert np.array_equal(depth.cpu().numpy(), d_ref)
+    ref, l1 = orc.scan(p_ref, s_ref, d_ref, q.cpu().numpy(), w.n)
+    assert_scores_close(sc.cpu().numpy(), ref, l1)
+
+
+@pytest.mark.parametrize("budget", [0, 1, 7, 48, 68, 92, 136, 300, 512])
+def test_plan_bit_exact(fathom_gpu, orc, budget):
+    w = dataclasses.replace(inputs.LAYER_32K, H=16, n=4096, seed=21)
+    k, q, s2 = make(w)
+    depth, active, na, theta = fathom_gpu.plan(s2, q, budget)
+    torch.cuda.synchronize()
+    d_ref, a_ref, na_ref, th_ref = orc.plan(s2.cpu().numpy(), q.cpu().numpy(), budget)
+    assert np.array_equal(depth.cpu().numpy(), d_ref)
+    assert np.array_equal(np_u16(active), a_ref)
+    assert np.array_equal(na.cpu().numpy(), na_ref)
+    assert np.array_equal(theta.cpu().numpy(), th_ref.astype(np.float32))
+
+
+def test_plan_per_group_budgets_and_edge_importances(fathom_gpu, orc):
+    rng = np.random.default_rng(0)
+    H, G, D = 12, 4, 128
+    q = rng.standard_normal((H, G, D)).astype(np.float32)
+    s2 = np.abs(rng.standard_normal((H, D))).astype(np.float32)
+    s2[0, :] = 1.0; q[0] = 1.0                        # all importances tied
+    s2[1, :64] = 0.0                                  # half the channels worthless
+    s2[2] = np.float32(1e-42) * (1 + np.arange(D))    # subnormal importances
+    q[3, :, ::2] = 0.0
+    s2[4] = np.exp(rng.uniform(-80, 80, D)).astype(np.float32)   # wide dynamic range
+    budgets = np.array([5, 48, 100, 48, 136, 0, 512, 1, 47, 49, 255, 256], np.int32)
+    depth, active, na, theta = fathom_gpu.plan(torch.tensor(s2, device=DEV), torch.tensor(q, device=DEV),
+                                               torch.tensor(budgets, device=DEV))
+    torch.cuda.synchronize()
+    d_ref, a_ref, na_ref, th_ref = orc.plan(s2, q, budgets)
+    assert np.array_equal(depth.cpu().numpy(), d_ref)
+    assert np.array_equal(np_u16(active), a_ref)
+    assert np.array_equal(na.cpu().numpy(), na_ref)
+
+
+@pytest.mark.parametrize("r", [0, 1, 16, 32, 128])
+def test_plan_fixed_bit_exact(fathom_gpu, orc, r):
+    w = dataclasses.replace(inputs.LAYER_32K, H=16, n=4096, seed=22)
+    _, q, _ = make(w)
+    q[3, :, 7] = q[3, :, 9]  # a tie, broken towards the lower channel
+    depth, active, na = fathom_gpu.plan_fixed(q, r)
+    torch.cuda.synchronize()
+    d_ref, a_ref, na_ref = orc.plan_fixed(q.cpu().numpy(), r)
+    assert np.array_equal(depth.cpu().numpy(), d_ref)
+    assert np.array_equal(np_u16(active), a_ref)
+    assert np.array_equal(na.cpu().numpy(), na_ref)
+
+
+def _full_path(fathom_gpu, orc, w, budget, fixed_r=None):
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    if fixed_r is None:
+        depth, active, na, _ = fathom_gpu.plan(s2, q, budget)
+    else:
+        depth, active, na = fathom_gpu.plan_fixed(q, fixed_r)
+    sc = fathom_gpu.scan(planes, scales, w.n, active, na, q)
+    idx, uni, cnt = fathom_gpu.topk(w.H, w.G, w.n, w.k, scores=sc)
+    torch.cuda.synchronize()
+    p_ref, s_ref = oracle_pack(orc, k, planes.shape[-1])
+    assert np.array_equal(np_u64(planes), p_ref) and np.array_equal(np_u16(scales), s_ref)
+    qn = q.cpu().numpy()
+    if fixed_r is None:
+        d_ref = orc.plan(s2.cpu().numpy(), qn, budget)[0]
+    else:
+        d_ref = orc.plan_fixed(qn, fixed_r)[0]
+    assert np.array_equal(depth.cpu().numpy(), d_ref)
+    ref, l1 = orc.scan(p_ref, s_ref, d_ref, qn, w.n)
+    gsc = sc.cpu().numpy()
+    assert_scores_close(gsc, ref, l1)
+    gidx = idx.cpu().numpy()
+    # exact against a full sort of the GPU's own fp32 scores
+    for h in range(w.H):
+        for g in range(w.G):
+            assert np.array_equal(gidx[h, g], lexsort_topk(gsc[h, g], w.k))
+    # up to ties against the oracle's fp64 top-k
+    r_idx, r_uni, r_cnt = orc.topk(ref, w.k)
+    assert_topk_sets_match(gidx, r_idx, ref, l1, w.k)
+    # union = sorted unique of the GPU's own lists
+    guni, gcnt = uni.cpu().numpy(), cnt.cpu().numpy()
+    for h in range(w.H):
+        u = np.unique(gidx[h].reshape(-1))
+        assert gcnt[h] == len(u)
+        assert np.array_equal(guni[h, :gcnt[h]], u) and np.all(guni[h, gcnt[h]:] == -1)
+    return planes, scales, active, na, q, sc, idx, uni, cnt
+
+
+def test_tiny_full_path(fathom_gpu, orc):
+    _full_path(fathom_gpu, orc, inputs.TINY, 48)
+
+
+@pytest.mark.parametrize("budget", [48, 68, 92, 136])
+def test_layer_32k_full_path(fathom_gpu, orc, budget):
+    _full_path(fathom_gpu, orc, inputs.LAYER_32K, budget)
+
+
+def test_layer_32k_fixed_136_bit_scan(fathom_gpu, orc):
+    _full_path(fathom_gpu, orc, inputs.LAYER_32K, None, fixed_r=32)
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (37, 37), (64, 5), (5037, 1), (5037, 100)])
+def test_ragged_and_degenerate_sizes(fathom_gpu, orc, n, k):
+    w = dataclasses.replace(inputs.TINY, name=f"n{n}", H=2, n=n, k=k, n_cal=n, seed=30 + n)
+    _full_path(fathom_gpu, orc, w, 48)
+
+
+def test_zero_budget_all_scores_zero_topk_takes_lowest_indices(fathom_gpu, orc):
+    w = dataclasses.replace(inputs.TINY, H=2, n=3000, k=50, seed=40)
+    *_, sc, idx, uni, cnt = _full_path(fathom_gpu, orc, w, 0)
+    assert torch.all(sc == 0)
+    assert np.array_equal(idx.cpu().numpy()[0, 0], np.arange(50))
+
+
+@pytest.mark.parametrize("budget", [48, 136])
+def test_candidate_path_equals_dense(fathom_gpu, orc, budget):
+    w = inputs.LAYER_32K
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    depth, active, na, _ = fathom_gpu.plan(s2, q, budget)
+    dense = fathom_gpu.scan(planes, scales, w.n, active, na, q)
+    d_idx, d_uni, d_cnt = fathom_gpu.topk(w.H, w.G, w.n, w.k, scores=dense)
+    step = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, budget=budget)
+    c_idx, c_uni, c_cnt = step.run(q, check_overflow=False)
+    torch.cuda.synchronize()
+    assert torch.all(c_cnt >= 0)   # every group proved exact without a rerun
+    assert torch.equal(c_idx, d_idx) and torch.equal(c_uni, d_uni) and torch.equal(c_cnt, d_cnt)
+
+
+def test_candidate_overflow_is_flagged_and_repaired(fathom_gpu, orc):
+    # Budget 0: every score is 0, so every key reaches the sampled threshold
+    # and the candidate buffer overflows; the group must be flagged, and the
+    # dense rerun must give the dense answer.
+    w = dataclasses.replace(inputs.LAYER_32K, H=2, seed=41)
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    step = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, budget=0)
+    step.run_plan(q)
+    step.run_scan(q)
+    idx, uni, cnt = step.run_topk()
+    torch.cuda.synchronize()
+    assert torch.all(cnt == fathom_gpu.ERR_OVERFLOW)
+    assert step.repair(q) == 2
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy()[1, 3], np.arange(w.k))
+    assert torch.all(cnt == w.k)
