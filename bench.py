@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the Fathom decode-step key scan on B200.
+
+One step = the per-decode-step hot path over a resident bit-plane index:
+plan (reverse water-filling) -> threshold pre-pass -> variable-depth
+candidate scan -> radix top-k per query head -> union per KV head, for all
+layer-head groups of the workload.  The index is built once (prefill,
+``fathom_pack``) before timing; its build is timed separately and reported
+under ``pack``.
+
+Default workload: Qwen3-8B-shaped decode step at 1M tokens -- 36 layers x 8
+KV heads = 288 groups, 128 channels, 4 query heads per group, 48 plane bits
+per token, k = 512.  Keys, queries and sigma^2 are seeded synthetic data
+(``long_context_decode_bit_b200.inputs``).  The 20.5 GB index is far larger
+than L2, so no flush is needed between steps.
+
+``--impl reference`` times the CPU oracle (test infrastructure) on the
+host cores instead, on a bounded sample of the same workload.
+
+Under torchrun every rank runs its own full workload (independent
+sessions, weak scaling); only timing is reduced across ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "keys scanned/s & scan GB/s vs HBM peak, 288 layer-heads @1M ctx, 48-bit"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("fathom", "reference"), default="fathom")
+    ap.add_argument("--workload", default="qwen3-8b-step-288x1048576")
+    ap.add_argument("--budget", type=int, default=48)
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--no-sweep", action="store_true", help="skip the budget / per-layer sweep")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--cpu-groups", type=int, default=1, help="groups in the CPU-oracle sample")
+    ap.add_argument("--quiet", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (host logic; covered by tests with gloo on CPU)
+# ----------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def rank_workload(w, rank: int):
+    """Each rank scans its own independent sessions: same shapes, own seed."""
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def reduce_max(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# clocks, peaks, profile-derived traffic
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("scan.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "long_context_decode_bit_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, budget: int):
+    """DRAM bytes per launch of the filter scan from a committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "scan_filter_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = d.get(f"{workload}@{budget}")
+    if not ent or ent.get("kernel_sha") != kernel_source_sha():
+        return None
+    return float(ent["dram_bytes_per_launch"])
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+def build_index(w, device, chunk: int = 8, log=print):
+    """Generate keys per chunk of groups and pack them at once (the raw keys
+    of the full workload would not fit).  Returns planes, scales, sigma2, q
+    and the pack timing of the first chunk."""
+    import torch
+    from long_context_decode_bit_b200 import fathom, inputs
+    nbs = fathom.nb_stride(w.n)
+    planes = torch.zeros((w.H, w.D, 4, nbs), dtype=torch.int64, device=device)
+    scales = torch.zeros((w.H, w.D, nbs), dtype=torch.int16, device=device)
+    sigma2 = torch.empty((w.H, w.D), dtype=torch.float32, device=device)
+    pack_ms = None
+    for h0 in range(0, w.H, chunk):
+        h1 = min(w.H, h0 + chunk)
+        keys = inputs.keys(w, h0, h1, device=device)
+        sigma2[h0:h1] = inputs.calibration_sigma2(keys, w.n_cal)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fathom.pack(keys, planes=planes[h0:h1], scales=scales[h0:h1])
+        e1.record()
+        if pack_ms is None:
+            torch.cuda.synchronize()
+            pack_ms = (e0.elapsed_time(e1), h1 - h0, keys.numel() * keys.element_size())
+        del keys
+    q = inputs.queries(w, 0, w.H, device=device).float().contiguous()
+    torch.cuda.synchronize()
+    ms, groups, kbytes = pack_ms
+    out_bytes = groups * w.D * (4 * 8 + 2) * w.nb
+    pack = {"ms_per_group": ms / groups, "keys_GBps": kbytes / ms / 1e6,
+            "traffic_GBps": (kbytes + out_bytes) / ms / 1e6, "groups_timed": groups}
+    return planes, scales, sigma2, q, pack
+
+
+def plan_bytes(step, w):
+    """Algorithmic bytes of one filter scan: per group n*sum(t)/8 plane bytes,
+    2 bytes per active channel per 64-token block, and the fp32 queries."""
+    from long_context_decode_bit_b200 import accounting
+    depth, _, n_active, _ = step.plan_out
+    bits = depth.to("cpu").int().sum(dim=1).tolist()
+    na = n_active.to("cpu").tolist()
+    return accounting.step_scan_bytes(w.n, bits, na, w.G, w.D), bits, na
+
+
+def time_steps(step_fn, steps, warmup, device, kernel_events=False):
+    import torch
+    for _ in range(warmup):
+        step_fn(None)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for i in range(steps):
+        step_fn(pairs[i])
+    s1.record()
+    torch.cuda.synchronize(device)
+    total_ms = s0.elapsed_time(s1)
+    kern_ms = [a.elapsed_time(b) for a, b in pairs] if kernel_events else []
+    barrier(device)
+    return total_ms, kern_ms
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from long_context_decode_bit_b200 import fathom, inputs
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    log = (lambda *a: print(*a, file=sys.stderr, flush=True)) if (rank == 0 and not args.quiet) else (lambda *a: None)
+    fathom.load()
+
+    base = inputs.WORKLOADS[args.workload]
+    if args.k is not None:
+        base = dataclasses.replace(base, k=args.k)
+    w = rank_workload(base, rank)
+    B, k = args.budget, w.k
+    t0 = time.time()
+    planes, scales, sigma2, q, pack = build_index(w, device, log=log)
+    log(f"[bench] index built in {time.time() - t0:.1f}s: {w.H} groups x {w.n} tokens, "
+        f"{(planes.numel() * 8 + scales.numel() * 2) / 1e9:.2f} GB")
+
+    step = fathom.Step(planes, scales, w.n, sigma2, w.G, k, budget=B)
+    launches_per_step = 6   # plan, sample scan, tau, filter scan, top-k, union
+
+    def one(ev):
+        step.run_plan(q)
+        step.run_prepare(q)
+        if ev is not None:
+            ev[0].record()
+        step.run_filter(q)
+        if ev is not None:
+            ev[1].record()
+        step.run_topk()
+
+    # Warm up once and make sure no group needs the dense rerun.
+    one(None)
+    torch.cuda.synchronize(device)
+    fallback = step.repair(q)
+    if fallback:
+        log(f"[bench] {fallback} groups overflowed the candidate pass; their dense rerun is timed")
+
+        def one(ev, _inner=one):  # noqa: F811
+            _inner(ev)
+            step.repair(q)
+
+    alg_bytes, bits, na = plan_bytes(step, w)
+    props = torch.cuda.get_device_properties(device)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    with ClockSampler(gpu_id) as clk:
+        total_ms, filt_ms = time_steps(one, args.steps, args.warmup, device, kernel_events=True)
+    clocks = clk.summary()
+    idx, uni, cnt = step.topk_out
+    bad_after = int((cnt < 0).sum().item())
+    total_ms = reduce_max(total_ms, device)
+    filt_mean = reduce_max(statistics.fmean(filt_ms), device)
+    ms_per_step = total_ms / args.steps
+    keys_per_step = world * w.H * w.n
+    value = keys_per_step / (ms_per_step / 1e3)
+    peak, peak_src = measured_peaks()
+    achieved = alg_bytes / (filt_mean / 1e3) / 1e9
+    traffic = profiled_traffic(base.name, B)
+
+    # End to end through the public API: per step, queries H2D from pinned
+    # host memory, the step, and its results D2H into pinned host memory.
+    q_host = q.to("cpu").pin_memory()
+    q_dev = torch.empty_like(q)
+    res_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in step.topk_out]
+
+    def e2e_step(_):
+        q_dev.copy_(q_host, non_blocking=True)
+        step.run_plan(q_dev)
+        step.run_prepare(q_dev)
+        step.run_filter(q_dev)
+        step.run_topk()
+        for hsrc, dev_t in zip(res_host, step.topk_out):
+            hsrc.copy_(dev_t, non_blocking=True)
+        torch.cuda.synchronize(device)
+        if bool((res_host[2] < 0).any()):
+            step.repair(q_dev)
+            for hsrc, dev_t in zip(res_host, step.topk_out):
+                hsrc.copy_(dev_t, non_blocking=True)
+            torch.cuda.synchronize(device)
+
+    e2e_ms, _ = time_steps(e2e_step, args.steps, max(3, args.warmup // 2), device)
+    e2e_ms = reduce_max(e2e_ms, device) / args.steps
+    h2d = q_host.numel() * q_host.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in res_host)
+
+    sweep = None
+    if not args.no_sweep:
+        sweep = run_sweep(w, planes, scales, sigma2, q, k, device, log)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": base.name, "layer_heads": w.H, "n": w.n, "head_dim": w.D, "gqa": w.G,
+                   "budget_bits": B, "k": k, "key_dtype": "bf16", "basis": "raw",
+                   "parallelism": "weak: independent sessions per GPU" if world > 1 else "single GPU",
+                   "l2": "no flush: the 20 GB index is read once per step, far above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": "scan_kernel<4> (FILTER)",
+                     "peak_source": f"{peak_src} hbm_gbs (copy)"},
+        "scan": {"ms": filt_mean, "GBps": achieved, "alg_bytes": alg_bytes,
+                 "read_bits_per_token": alg_bytes * 8 / (w.H * w.n),
+                 "plane_bits_mean": statistics.fmean(bits), "active_channels_mean": statistics.fmean(na),
+                 "active_channels_range": [min(na), max(na)]},
+        "e2e": {"value": keys_per_step / (e2e_ms / 1e3), "unit": "keys/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps + (2 * fallback * args.steps if fallback else 0),
+        "clocks": clocks, "pack": pack, "fallback_groups": fallback, "overflow_after_timing": bad_after,
+    }
+    if sweep is not None:
+        result["sweep"] = sweep
+    if rank == 0 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(w, k, B, args.cpu_groups, device, log)
+    if world > 1:
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+def run_sweep(w, planes, scales, sigma2, q, k, device, log):
+    """Step time at other budgets, the fixed 136-bit scan on the same data,
+    and the layer-sequential launch pattern (36 x 8 groups)."""
+    import torch
+    from long_context_decode_bit_b200 import fathom
+    out = {}
+    variants = [(f"B{b}", dict(budget=b)) for b in (48, 68, 92, 136)] + [("fixed136_r32", dict(fixed_r=32))]
+    for name, kw in variants:
+        st = fathom.Step(planes, scales, w.n, sigma2, w.G, k, **kw)
+
+        def one(ev, st=st):
+            st.run_plan(q)
+            st.run_prepare(q)
+            if ev is not None:
+                ev[0].record()
+            st.run_filter(q)
+            if ev is not None:
+                ev[1].record()
+            st.run_topk()
+        one(None)
+        torch.cuda.synchronize(device)
+        fb = st.repair(q)
+        alg, bits, na = plan_bytes(st, w)
+        tot, fk = time_steps(one, 5, 2, device, kernel_events=True)
+        fm = statistics.fmean(fk)
+        out[name] = {"ms_per_step": tot / 5, "scan_ms": fm, "scan_GBps": alg / (fm / 1e3) / 1e9,
+                     "read_bits_per_token": alg * 8 / (w.H * w.n), "plane_bits_mean": statistics.fmean(bits),
+                     "active_channels_mean": statistics.fmean(na), "fallback_groups": fb}
+        del st
+    layers = w.H // 8 if w.H % 8 == 0 else 1
+    per = w.H // layers
+    steps = [fathom.Step(planes[l * per:(l + 1) * per], scales[l * per:(l + 1) * per], w.n,
+                         sigma2[l * per:(l + 1) * per], w.G, k, budget=48) for l in range(layers)]
+    qs = [q[l * per:(l + 1) * per] for l in range(layers)]
+
+    def seq(ev):
+        for st, ql in zip(steps, qs):
+            st.run(ql, check_overflow=False)
+    seq(None)
+    tot, _ = time_steps(seq, 5, 2, device)
+    out["per_layer_B48"] = {"layers": layers, "groups_per_layer": per, "ms_per_step": tot / 5}
+    return out
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+def _oracle_sample(w, groups: int, device):
+    import numpy as np
+    import torch
+    import oracle
+    from long_context_decode_bit_b200 import inputs
+    k = inputs.keys(w, 0, groups, device=device)
+    s2 = inputs.calibration_sigma2(k, w.n_cal).cpu().numpy()
+    qn = inputs.queries(w, 0, groups, device=device).float().cpu().numpy()
+    kn = k.contiguous().view(torch.int16).cpu().numpy().view(np.uint16) if k.dtype == torch.bfloat16 \
+        else k.cpu().numpy()
+    del k
+    planes, scales = oracle.pack(kn)
+    return planes, scales, s2, qn
+
+
+def _oracle_step(planes, scales, s2, qn, n, B, k):
+    import oracle
+    depth = oracle.plan(s2, qn, B)[0]
+    sc = oracle.scan(planes, scales, depth, qn, n, with_l1=False)
+    oracle.topk(sc, k)
+
+
+def cpu_baseline(w, k, B, groups, device, log):
+    planes, scales, s2, qn = _oracle_sample(w, groups, device)
+    t = time.perf_counter()
+    _oracle_step(planes, scales, s2, qn, w.n, B, k)
+    dt = time.perf_counter() - t
+    log(f"[bench] CPU oracle: {groups} group(s) x {w.n} keys in {dt:.1f}s")
+    return {"value": groups * w.n / dt, "unit": "keys/s", "cores": 1, "kind": "oracle",
+            "sample": f"{groups} of {w.H} groups at full length n={w.n}: plan + fp64 scan + full-sort top-k "
+                      f"+ union, single-threaded C oracle, keys prepacked by the oracle outside the timed region"}
+
+
+def run_reference(args):
+    import torch
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    from long_context_decode_bit_b200 import inputs
+    base = inputs.WORKLOADS[args.workload]
+    if args.k is not None:
+        base = dataclasses.replace(base, k=args.k)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    groups = max(1, args.cpu_groups)
+    planes, scales, s2, qn = _oracle_sample(base, groups, dev)
+    for _ in range(args.warmup):
+        _oracle_step(planes, scales, s2, qn, base.n, args.budget, base.k)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(planes, scales, s2, qn, base.n, args.budget, base.k)
+    dt = (time.perf_counter() - t) / args.steps
+    value = groups * base.n / dt
+    sample = (f"each step: {groups} of {base.H} groups at full length n={base.n} (plan + fp64 scan + full-sort "
+              f"top-k + union), single-threaded C oracle")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": base.name, "layer_heads": base.H, "n": base.n, "head_dim": base.D,
+                       "gqa": base.G, "budget_bits": args.budget, "k": base.k},
+            "cpu_baseline": {"value": value, "unit": "keys/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -57,7 +57,9 @@ typedef struct CUstream_st* fathom_stream_t; /* same type as cudaStream_t */
 
 /* Output modes of fathom_scan. */
 #define FATHOM_SCAN_DENSE 0
-#define FATHOM_SCAN_CANDIDATE 1
+#define FATHOM_SCAN_CANDIDATE 1 /* PREPARE then FILTER, in one call */
+#define FATHOM_SCAN_PREPARE 2   /* threshold pass only */
+#define FATHOM_SCAN_FILTER 3    /* main candidate pass only, after PREPARE */
 
 /* Library version as 10000*major + 100*minor + patch. */
 int fathom_version(void);
@@ -188,10 +190,17 @@ size_t fathom_scan_cand_bytes(int64_t H, int G, int64_t n, int k);
  *                   filter only: fathom_topk checks that at least k keys
  *                   passed and none were dropped, which proves the top-k
  *                   exact, and flags the group otherwise.
+ *                   FATHOM_SCAN_PREPARE: only the threshold part (sample
+ *                   pass, tau per head, counters reset to 0).
+ *                   FATHOM_SCAN_FILTER: only the main pass, appending to a
+ *                   cand buffer that a PREPARE call with the same H, G, n, k
+ *                   readied earlier on the stream.  CANDIDATE is PREPARE
+ *                   followed by FILTER; the split lets a caller time or
+ *                   overlap the two.
  *   scores          DEVICE out, fp32 [H][G][n] (DENSE; ignored otherwise).
  *   cand, cand_bytes  DEVICE scratch/out of at least
- *                   fathom_scan_cand_bytes(H, G, n, k) bytes (CANDIDATE;
- *                   ignored in DENSE mode), 16-byte aligned.
+ *                   fathom_scan_cand_bytes(H, G, n, k) bytes (all modes but
+ *                   DENSE, which ignores it), 16-byte aligned.
  *   k               winners per query head that will be asked of
  *                   fathom_topk (sizes the candidate pass).
  */

@@ -162,7 +162,7 @@ int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
 {
     if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
-    if (mode != FATHOM_SCAN_DENSE && mode != FATHOM_SCAN_CANDIDATE) return FATHOM_ERR_INVALID_ARG;
+    if (mode < FATHOM_SCAN_DENSE || mode > FATHOM_SCAN_FILTER) return FATHOM_ERR_INVALID_ARG;
     if (H == 0 || n == 0) return FATHOM_OK;
     const int64_t nb = ceil_div(n, kBlockTokens);
     if (nb_stride < nb) return FATHOM_ERR_INVALID_ARG;

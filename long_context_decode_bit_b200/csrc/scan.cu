@@ -315,14 +315,16 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
     a.entries = reinterpret_cast<int2*>(base + L.off_entries);
     a.cap = L.cap;
     a.n_sample = L.n_sample;
-    if (L.sample_tiles > 0) {
-        a.mode = kSample;
-        a.tile_stride = L.tile_stride;
-        int st = launch_scan_mode(a, G, static_cast<unsigned>(L.sample_tiles), static_cast<unsigned>(H), stream);
-        if (st) return st;
+    if (mode == FATHOM_SCAN_CANDIDATE || mode == FATHOM_SCAN_PREPARE) {
+        if (L.sample_tiles > 0) {
+            a.mode = kSample;
+            a.tile_stride = L.tile_stride;
+            int st = launch_scan_mode(a, G, static_cast<unsigned>(L.sample_tiles), static_cast<unsigned>(H), stream);
+            if (st) return st;
+        }
+        int st = launch_tau(a.sample, a.hdr, L.heads, L.n_sample, L.m_rank, stream);
+        if (st || mode == FATHOM_SCAN_PREPARE) return st;
     }
-    int st = launch_tau(a.sample, a.hdr, L.heads, L.n_sample, L.m_rank, stream);
-    if (st) return st;
     a.mode = kCandidate;
     a.tile_stride = 1;
     return launch_scan_mode(a, G, tiles, static_cast<unsigned>(H), stream);

@@ -28,6 +28,8 @@ KEYS_F32 = 0
 KEYS_BF16 = 1
 SCAN_DENSE = 0
 SCAN_CANDIDATE = 1
+SCAN_PREPARE = 2
+SCAN_FILTER = 3
 
 # Every symbol include/fathom.h declares.
 EXPORTS = (
@@ -173,7 +175,7 @@ def scan(planes, scales, n: int, active, n_active, q, mode: int = SCAN_DENSE, k:
     if cand is None:
         cand = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     _check(lib().fathom_scan(_p(planes), _p(scales), H, D, n, nbs, _p(active), _p(n_active), _p(q), G,
-                             SCAN_CANDIDATE, None, _p(cand), cand.numel() * cand.element_size(), int(k),
+                             int(mode), None, _p(cand), cand.numel() * cand.element_size(), int(k),
                              _stream(stream)), "fathom_scan")
     return cand
 
@@ -227,9 +229,17 @@ class Step:
             plan_fixed(q, self.fixed_r, out=self.plan_out[:3])
         return self.plan_out
 
-    def run_scan(self, q):
+    def run_prepare(self, q):
         _, active, n_active, _ = self.plan_out
-        return scan(self.planes, self.scales, self.n, active, n_active, q, SCAN_CANDIDATE, self.k, cand=self.cand)
+        return scan(self.planes, self.scales, self.n, active, n_active, q, SCAN_PREPARE, self.k, cand=self.cand)
+
+    def run_filter(self, q):
+        _, active, n_active, _ = self.plan_out
+        return scan(self.planes, self.scales, self.n, active, n_active, q, SCAN_FILTER, self.k, cand=self.cand)
+
+    def run_scan(self, q):
+        self.run_prepare(q)
+        return self.run_filter(q)
 
     def run_topk(self):
         return topk(self.H, self.G, self.n, self.k, cand=self.cand, out=self.topk_out)
