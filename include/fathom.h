@@ -240,6 +240,44 @@ int fathom_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
                 int32_t* idx, int32_t* union_idx, int32_t* union_count,
                 void* workspace, size_t ws_bytes, fathom_stream_t stream);
 
+/*
+ * fathom_scan_topk_noalloc -- fathom_scan in CANDIDATE mode followed by
+ * fathom_topk, for callers that cannot allocate device memory.  (The paper
+ * has no counterpart: this is a deployment convenience of this library.)
+ *
+ * Some callers cannot hand the scan a scratch buffer: an operator plugged
+ * into another inference runtime that has already reserved the free device
+ * memory for its KV-cache pool and gives the operator no allocator, or a
+ * decode loop that must not call cudaMalloc because it synchronises the
+ * device.  This call keeps the candidate buffer in an array that the
+ * library itself owns in device memory, of FATHOM_NOALLOC_SCRATCH_BYTES;
+ * every device that loads the library holds that much until the process
+ * exits.  Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ *
+ * Arguments and results are those of fathom_scan (without mode, scores,
+ * cand, cand_bytes) and of fathom_topk (without scores, cand, workspace):
+ * union_count[h] == FATHOM_ERR_OVERFLOW still marks a group to rerun densely.
+ * Sizes whose candidate buffer, fathom_scan_cand_bytes(H, G, n, k), exceeds
+ * FATHOM_NOALLOC_SCRATCH_BYTES are rejected with FATHOM_ERR_WORKSPACE
+ * before anything is launched (one layer of 8 KV heads with G = 4, k = 512
+ * fits at n = 1M; a whole 288-group step does not -- call it per layer).
+ *
+ * The first call on a device looks up the array's device address (a
+ * one-time cudaGetSymbolAddress with that device current); make that first
+ * call before any stream capture.  All calls share the one array, and each
+ * call's threshold pass resets the counters it uses, so leftover contents
+ * never leak into a result; but calls whose work overlaps on the GPU (two
+ * streams, or two threads on one device) race on the array and must be
+ * serialised by the caller.
+ */
+#define FATHOM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+int fathom_scan_topk_noalloc(const uint64_t* planes, const uint16_t* scales, int64_t H, int D,
+                             int64_t n, int64_t nb_stride, const uint16_t* active,
+                             const int32_t* n_active, const float* q, int G, int k,
+                             int32_t* idx, int32_t* union_idx, int32_t* union_count,
+                             fathom_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -35,8 +35,10 @@ SCAN_FILTER = 3
 EXPORTS = (
     "fathom_version", "fathom_status_string", "fathom_last_cuda_error", "fathom_nb_stride",
     "fathom_pack", "fathom_plan", "fathom_plan_fixed", "fathom_scan_cand_bytes", "fathom_scan",
-    "fathom_topk_workspace_bytes", "fathom_topk",
+    "fathom_topk_workspace_bytes", "fathom_topk", "fathom_scan_topk_noalloc",
 )
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _lib = None
 
@@ -72,6 +74,7 @@ def load(path: str = LIB_PATH):
         "fathom_scan": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, SZ, I, P]),
         "fathom_topk_workspace_bytes": (SZ, [I64, I, I64, I]),
         "fathom_topk": (I, [P, P, I64, I, I64, I, P, P, P, P, SZ, P]),
+        "fathom_scan_topk_noalloc": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -195,6 +198,24 @@ def topk(H: int, G: int, n: int, k: int, scores=None, cand=None, out=None, works
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().fathom_topk(_p(scores), _p(cand), H, G, n, int(k), _p(idx), _p(uni), _p(cnt), _p(workspace),
                              ws_bytes, _stream(stream)), "fathom_topk")
+    return idx, uni, cnt
+
+
+def scan_topk_noalloc(planes, scales, n: int, active, n_active, q, k: int, out=None, stream=None):
+    """Candidate scan + top-k + union using the library's own fixed device
+    scratch instead of a caller buffer, for callers that cannot allocate
+    device memory (see fathom_scan_topk_noalloc in include/fathom.h).  The
+    output tensors may be preallocated and passed as ``out``."""
+    H, G, D = q.shape
+    if out is None:
+        dev = q.device
+        out = (torch.empty((H, G, k), dtype=torch.int32, device=dev),
+               torch.empty((H, G * k), dtype=torch.int32, device=dev),
+               torch.empty(H, dtype=torch.int32, device=dev))
+    idx, uni, cnt = out
+    _check(lib().fathom_scan_topk_noalloc(_p(planes), _p(scales), H, D, n, planes.shape[-1], _p(active),
+                                          _p(n_active), _p(q), G, int(k), _p(idx), _p(uni), _p(cnt),
+                                          _stream(stream)), "fathom_scan_topk_noalloc")
     return idx, uni, cnt
 
 
