@@ -6,19 +6,28 @@
 // where c_t is the key's t-bit prefix code read from the first t plane rows
 // of channel j.  The K bytes are read once for all G heads.
 //
-// Work layout.  A CTA (4 warps) scores one tile of 16 consecutive 64-token
-// blocks of one group.  Active channels are processed in chunks of 32: the
-// chunk's plane rows (sum t words per block) and scale rows are staged in
-// shared memory with coalesced loads, then every lane scores four tokens of
-// one 32-bit half plane word at once:
-//   - token bits sit at positions l, l+8, l+16, l+24 of the half word
-//     (l = lane & 7); one funnel-shift rotation per plane moves plane p's
-//     four bits to bit 7-p of four different bytes, and one AND/OR merges
-//     them, so after t planes byte m holds c_t << (8 - t);
-//   - a byte permute drops byte m into the low mantissa bits of 1.5 * 2^23,
-//     and one FMA with exact constants turns that float into the odd
-//     integer 2 c_t - 2^t + 1;
-//   - G FMAs per token add coefficient (q_{g,j} 2^-t) * s_{b,j} times it.
+// Work layout.  A CTA (4 warps) walks `tiles_per_cta` consecutive tiles of
+// 16 64-token blocks of one group.  Each warp owns 4 blocks of a tile; a
+// lane owns 8 tokens of one block: bit positions l, l+8, l+16, l+24
+// (l = lane & 7) of the block's low and of its high 32-bit plane half.
+//
+// Per tile, the active channels (sorted by depth once per CTA) are staged
+// in chunks: their plane words go to shared memory with cp.async, laid out
+// [block][slot][64-bit word] so that a lane fetches all planes of a channel
+// with one or two 128-bit loads; the coefficients (q_{g,j} 2^-t) * s_{b,j}
+// of every (channel, block) are computed once into shared memory as
+// duplicated pairs for the packed fp32x2 FMA.
+//
+// Decoding, per channel and per 32-bit half (four tokens at once):
+//   - depth 1: one shift moves each token's sign bit to bit 7 of its own
+//     byte, one AND/XOR turns the bytes into 0x3F / 0xBF, and one byte
+//     permute per token lays that byte over 0x00800000: +-1.0f exactly.
+//   - depth t >= 2: one funnel-shift rotation per plane moves plane p's
+//     four bits to bit 7-p of four bytes and one AND/OR merges them, so
+//     byte m holds c_t << (8-t); a byte permute drops it into the low
+//     mantissa of 1.5 * 2^23 and one packed FMA with exact constants gives
+//     the odd integers 2 c_t - 2^t + 1 of two tokens.
+//   - then G packed FMAs per token pair add coefficient * value.
 // There are no tensor cores: the contraction is a gathered, variable-depth
 // GEMV whose operand must be decoded bit by bit first.
 //
@@ -34,10 +43,10 @@ namespace {
 
 constexpr int kScanThreads = 128;
 constexpr int kScanWarps = kScanThreads / 32;
-constexpr int kChunkCh = 32;                     // active channels per staging chunk
-constexpr int kChunkRows = kChunkCh * kPlanes;   // plane rows per chunk (max)
 constexpr int kBlocksPerWarp = kScanTileBlocks / kScanWarps;  // 4
-constexpr int kSets = kBlocksPerWarp / 2;        // a lane set covers 2 blocks
+constexpr int kChunkCh = 40;        // channels per staging chunk
+constexpr int kChunkSlots = 64;     // 64-bit plane words per block per chunk
+constexpr int kWordStride = kChunkSlots * 8 + 16;  // bytes per staged block (+16 spreads banks)
 
 enum ScanMode { kDense = 0, kSample = 1, kCandidate = 2 };
 
@@ -53,200 +62,330 @@ struct ScanArgs {
     CandHeader* hdr;           // [H*G]
     float* sample;             // [H*G][n_sample]
     int2* entries;             // [H*G][cap]
-    int64_t cap, n_sample, tile_stride;
+    int64_t cap, n_sample, tile_stride, tiles;
+    int tiles_per_cta;
     int mode;
 };
 
+// Slots a channel of depth t takes in a staged block: depth 3 and 4 an
+// aligned 32-byte quad, depth 2 an aligned 16-byte pair, depth 1 one word.
+// Channels are staged in descending depth, so the alignment holds.
+__host__ __device__ constexpr int slots_of(int t) { return t >= 3 ? 4 : t; }
+
 template <int G>
-__global__ void __launch_bounds__(kScanThreads)
+struct SharedScan {
+    __align__(16) unsigned char words[kScanTileBlocks * kWordStride];
+    __align__(16) float2 coef[kChunkCh * kScanTileBlocks * G];   // duplicated pairs
+    float qs[kMaxD * G];             // q_{g,j} * 2^-t, depth-sorted order
+    uint16_t chan[kMaxD];            // depth-sorted entries j | t << 8
+    uint8_t slot[kMaxD];             // slot of each sorted channel within its chunk
+    int16_t chunk_begin[kMaxD + 1];  // chunk boundaries in sorted order
+    int16_t chunk_cnt[kMaxD][4];     // per chunk: channels of depth 4, 3, 2, 1
+    int n_chunks;
+    float tau[G];
+};
+
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem, bool valid)
+{
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    const int n = valid ? 8 : 0;   // 0: zero fill, nothing is read
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
+// Depth-1 values of the four tokens of one 32-bit half: +-1.0f.
+__device__ __forceinline__ void values_depth1(uint32_t w, int l, float2& v01, float2& v23)
+{
+    const uint32_t y = ((w << (7 - l)) & 0x80808080u) ^ 0xBFBFBFBFu;
+    v01.x = __uint_as_float(__byte_perm(y, 0x00800000u, 0x0654u));
+    v01.y = __uint_as_float(__byte_perm(y, 0x00800000u, 0x1654u));
+    v23.x = __uint_as_float(__byte_perm(y, 0x00800000u, 0x2654u));
+    v23.y = __uint_as_float(__byte_perm(y, 0x00800000u, 0x3654u));
+}
+
+// Depth-T (T >= 2) values of four tokens from T plane halves.
+template <int T>
+__device__ __forceinline__ void values_depth(const uint32_t (&w)[4], int l, float2& v01, float2& v23)
+{
+    uint32_t code = 0;
+#pragma unroll
+    for (int p = 0; p < T; ++p) {
+        const uint32_t x = __funnelshift_l(w[p], w[p], (7 - p - l) & 31);
+        code |= x & (0x01010101u << (7 - p));
+    }
+    constexpr float mul = static_cast<float>(1u << T) / 128.0f;                          // 2^(t-7)
+    constexpr float sub = 1.5f * static_cast<float>(1u << (16 + T)) + static_cast<float>((1u << T) - 1);
+    const float2 m2 = make_float2(mul, mul), s2 = make_float2(-sub, -sub);
+    float2 f01, f23;
+    f01.x = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7650u));
+    f01.y = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7651u));
+    f23.x = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7652u));
+    f23.y = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7653u));
+    v01 = __ffma2_rn(f01, m2, s2);   // exact odd integers
+    v23 = __ffma2_rn(f23, m2, s2);
+}
+
+// One channel of depth T for the lane's block: 8 tokens (4 pairs) x G heads.
+// c: index in depth-sorted order (selects the staged slot); cl: index within
+// the chunk (selects the coefficients).
+template <int G, int T>
+__device__ __forceinline__ void channel_step(const SharedScan<G>& S, int c, int cl, int blk, int l,
+                                             float2 (&acc)[4][G])
+{
+    const unsigned char* wrow = S.words + blk * kWordStride + S.slot[c] * 8;
+    uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
+    if (T == 1) {
+        const uint2 x = *reinterpret_cast<const uint2*>(wrow);
+        lo[0] = x.x; hi[0] = x.y;
+    } else {
+        const uint4 x = *reinterpret_cast<const uint4*>(wrow);
+        lo[0] = x.x; hi[0] = x.y; lo[1] = x.z; hi[1] = x.w;
+        if (T >= 3) {
+            const uint4 y = *reinterpret_cast<const uint4*>(wrow + 16);
+            lo[2] = y.x; hi[2] = y.y; lo[3] = y.z; hi[3] = y.w;
+        }
+    }
+    float2 v[4];
+    if (T == 1) {
+        values_depth1(lo[0], l, v[0], v[1]);
+        values_depth1(hi[0], l, v[2], v[3]);
+    } else {
+        values_depth<T>(lo, l, v[0], v[1]);
+        values_depth<T>(hi, l, v[2], v[3]);
+    }
+    const float2* cf = S.coef + (cl * kScanTileBlocks + blk) * G;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const float2 k2 = cf[g];
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) acc[pr][g] = __ffma2_rn(v[pr], k2, acc[pr][g]);
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kScanThreads, 4)
 scan_kernel(const ScanArgs a)
 {
-    __shared__ uint16_t act_s[kMaxD];
-    __shared__ float qs_s[kMaxD * G];
-    __shared__ uint16_t rowsrc_s[kChunkRows];       // (j << 2) | p per staged row
-    __shared__ __align__(16) uint64_t words_s[kChunkRows * kScanTileBlocks];
-    __shared__ uint16_t scale_s[kChunkCh * kScanTileBlocks];
-    __shared__ float tau_s[G];
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    SharedScan<G>& S = *reinterpret_cast<SharedScan<G>*>(smem_raw);
 
     const int64_t h = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int D = a.D;
     const int na = min(max(a.n_active[h], 0), D);   // trust nothing beyond D entries
-    const int64_t tile = static_cast<int64_t>(blockIdx.x) * a.tile_stride;
-    const int64_t b0 = tile * kScanTileBlocks;
 
-    // Plan of the group: active (j, t) and coefficients q_{g,j} * 2^-t.
-    for (int i = tid; i < na; i += kScanThreads) {
-        uint16_t e = a.active[h * D + i];
-        int j = e & 0xFF, t = min(e >> 8, kPlanes);
-        if (j >= D) t = 0;                  // malformed entry: read nothing
-        if (t == 0) j = 0;
-        e = static_cast<uint16_t>(j | (t << 8));
-        act_s[i] = e;
+    // ---- the group's plan, sorted by depth (4, 3, 2, 1), ascending j within a depth
+    if (tid < 32) {
+        int base = 0;
+        for (int t = 4; t >= 1; --t) {
+            for (int i0 = 0; i0 < na; i0 += 32) {
+                const int i = i0 + lane;
+                int j = 0, tt = 0;
+                if (i < na) {
+                    const uint16_t e = a.active[h * D + i];
+                    j = e & 0xFF;
+                    tt = min(e >> 8, kPlanes);
+                    if (j >= D) tt = 0;       // malformed entry: read nothing
+                }
+                const unsigned bal = __ballot_sync(0xffffffffu, tt == t);
+                if (tt == t) S.chan[base + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(j | (t << 8));
+                base += __popc(bal);
+            }
+        }
+        __syncwarp();
+        // Chunks of at most kChunkCh channels and kChunkSlots staged words.
+        if (lane == 0) {
+            int c = 0, k = 0;
+            while (c < base) {
+                S.chunk_begin[k] = static_cast<int16_t>(c);
+                int cnt[5] = {0, 0, 0, 0, 0}, slots = 0, ch = 0;
+                while (c < base && ch < kChunkCh) {
+                    const int t = S.chan[c] >> 8;
+                    if (slots + slots_of(t) > kChunkSlots) break;
+                    S.slot[c] = static_cast<uint8_t>(slots);
+                    slots += slots_of(t);
+                    cnt[t]++;
+                    ch++;
+                    c++;
+                }
+                S.chunk_cnt[k][0] = static_cast<int16_t>(cnt[4]);
+                S.chunk_cnt[k][1] = static_cast<int16_t>(cnt[3]);
+                S.chunk_cnt[k][2] = static_cast<int16_t>(cnt[2]);
+                S.chunk_cnt[k][3] = static_cast<int16_t>(cnt[1]);
+                k++;
+            }
+            S.chunk_begin[k] = static_cast<int16_t>(c);
+            S.n_chunks = k;
+        }
+    }
+    __syncthreads();
+    const int n_chunks = S.n_chunks;
+    const int nsorted = S.chunk_begin[n_chunks];
+    for (int i = tid; i < nsorted; i += kScanThreads) {
+        const int j = S.chan[i] & 0xFF, t = S.chan[i] >> 8;
         const float sc = __uint_as_float(static_cast<uint32_t>(127 - t) << 23);  // 2^-t
 #pragma unroll
-        for (int g = 0; g < G; ++g) qs_s[i * G + g] = __fmul_rn(a.q[(h * G + g) * D + j], sc);
+        for (int g = 0; g < G; ++g) S.qs[i * G + g] = __fmul_rn(a.q[(h * G + g) * D + j], sc);
     }
-    if (a.mode == kCandidate && tid < G) tau_s[tid] = a.hdr[h * G + tid].tau;
+    if (a.mode == kCandidate && tid < G) S.tau[tid] = a.hdr[h * G + tid].tau;
+    __syncthreads();   // qs and tau visible to every warp, even with no chunk to stage
 
-    // Lane geometry: which block of the warp's pair, which 32-bit half, and
-    // the bit offset l of its four tokens l, l+8, l+16, l+24.
-    const int blk_in_pair = lane >> 4;
-    const int half = (lane >> 3) & 1;
     const int l = lane & 7;
+    const int blk = warp * kBlocksPerWarp + (lane >> 3);   // the lane's block within a tile
 
-    float acc[kSets][4][G];
-#pragma unroll
-    for (int s = 0; s < kSets; ++s)
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-#pragma unroll
-            for (int g = 0; g < G; ++g) acc[s][m][g] = 0.0f;
+    for (int ti = 0; ti < a.tiles_per_cta; ++ti) {
+        const int64_t ltile = static_cast<int64_t>(blockIdx.x) * a.tiles_per_cta + ti;   // logical tile
+        if (ltile * a.tile_stride >= a.tiles) break;
+        const int64_t b0 = ltile * a.tile_stride * kScanTileBlocks;
 
-    __syncthreads();
+        float2 acc[4][G];
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr)
+#pragma unroll
+            for (int g = 0; g < G; ++g) acc[pr][g] = make_float2(0.0f, 0.0f);
 
-    const uint32_t* words32 = reinterpret_cast<const uint32_t*>(words_s);
-    for (int c0 = 0; c0 < na; c0 += kChunkCh) {
-        const int nc = min(kChunkCh, na - c0);
-        // Row table of the chunk: staged row r comes from plane (j, p).
-        if (tid == 0) {
-            int r = 0;
-            for (int c = 0; c < nc; ++c) {
-                const uint16_t e = act_s[c0 + c];
-                const int j = e & 0xFF, t = e >> 8;
-                for (int p = 0; p < t; ++p) rowsrc_s[r++] = static_cast<uint16_t>((j << 2) | p);
-            }
-        }
-        int rows = 0;
-        for (int c = 0; c < nc; ++c) rows += act_s[c0 + c] >> 8;
-        __syncthreads();
-
-        // Stage plane words: row r, block b at words_s[r * 16 + b].
-        for (int idx = tid; idx < rows * kScanTileBlocks; idx += kScanThreads) {
-            const int r = idx / kScanTileBlocks, b = idx % kScanTileBlocks;
-            const int src = rowsrc_s[r];
-            const int64_t row = (h * D + (src >> 2)) * kPlanes + (src & 3);
-            const int64_t blk = b0 + b;
-            words_s[r * kScanTileBlocks + b] = blk < a.nb ? __ldg(a.planes + row * a.nb_stride + blk) : 0ull;
-        }
-        for (int idx = tid; idx < nc * kScanTileBlocks; idx += kScanThreads) {
-            const int c = idx / kScanTileBlocks, b = idx % kScanTileBlocks;
-            const int j = act_s[c0 + c] & 0xFF;
-            const int64_t blk = b0 + b;
-            scale_s[c * kScanTileBlocks + b] = blk < a.nb ? __ldg(a.scales + (h * D + j) * a.nb_stride + blk) : 0;
-        }
-        __syncthreads();
-
-#pragma unroll
-        for (int s = 0; s < kSets; ++s) {
-            const int blk = warp * kBlocksPerWarp + s * 2 + blk_in_pair;   // block within tile
-            int row = 0;
-            for (int c = 0; c < nc; ++c) {
-                const int t = act_s[c0 + c] >> 8;
-                uint32_t code = 0;
-#pragma unroll
-                for (int p = 0; p < kPlanes; ++p) {
-                    if (p < t) {
-                        const uint32_t w = words32[(row + p) * (2 * kScanTileBlocks) + blk * 2 + half];
-                        const uint32_t x = __funnelshift_l(w, w, (7 - p - l) & 31);
-                        code |= x & (0x01010101u << (7 - p));
-                    }
-                }
-                row += t;
-                const float sblk = __half2float(__ushort_as_half(scale_s[c * kScanTileBlocks + blk]));
-                const float mul = __uint_as_float(static_cast<uint32_t>(120 + t) << 23);  // 2^(t-7)
-                const float sub = 1.5f * __uint_as_float(static_cast<uint32_t>(143 + t) << 23) +
-                                  static_cast<float>((1 << t) - 1);                    // 1.5*2^(16+t) + 2^t - 1
-                float coef[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) coef[g] = __fmul_rn(qs_s[(c0 + c) * G + g], sblk);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float f = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7650u + m));
-                    const float v = __fmaf_rn(f, mul, -sub);      // exact odd integer
-#pragma unroll
-                    for (int g = 0; g < G; ++g) acc[s][m][g] = __fmaf_rn(coef[g], v, acc[s][m][g]);
+        for (int ck = 0; ck < n_chunks; ++ck) {
+            const int c0 = S.chunk_begin[ck], c1 = S.chunk_begin[ck + 1];
+            __syncthreads();   // the previous chunk's buffers are free
+            // Stage plane words: 16 threads per channel, one block each.
+            {
+                const int b = tid & 15;
+                const int64_t blkg = b0 + b;
+                const bool valid = blkg < a.nb;
+                for (int c = c0 + (tid >> 4); c < c1; c += kScanThreads / 16) {
+                    const int j = S.chan[c] & 0xFF, t = S.chan[c] >> 8;
+                    const uint64_t* src = a.planes + (h * D + j) * kPlanes * a.nb_stride + (valid ? blkg : 0);
+                    unsigned char* dst = S.words + b * kWordStride + S.slot[c] * 8;
+                    for (int p = 0; p < t; ++p) cp_async8(dst + p * 8, src + p * a.nb_stride, valid);
                 }
             }
-        }
-        __syncthreads();
-    }
-
-    // Epilogue.
-    const int64_t tok_tile0 = b0 * kBlockTokens;
+            // Coefficients of every (channel, block), duplicated for the packed FMA.
+            for (int idx = tid; idx < (c1 - c0) * kScanTileBlocks; idx += kScanThreads) {
+                const int cl = idx / kScanTileBlocks, b = idx % kScanTileBlocks;
+                const int c = c0 + cl;
+                const int j = S.chan[c] & 0xFF;
+                const int64_t blkg = b0 + b;
+                const float s = blkg < a.nb ? __half2float(__ushort_as_half(
+                                                  __ldg(a.scales + (h * D + j) * a.nb_stride + blkg)))
+                                            : 0.0f;
+                float2* dst = S.coef + (cl * kScanTileBlocks + b) * G;
 #pragma unroll
-    for (int s = 0; s < kSets; ++s) {
-        const int blk = warp * kBlocksPerWarp + s * 2 + blk_in_pair;
-        const int local0 = blk * kBlockTokens + half * 32 + l;      // token within tile, m = 0
+                for (int g = 0; g < G; ++g) {
+                    const float v = __fmul_rn(S.qs[c * G + g], s);
+                    dst[g] = make_float2(v, v);
+                }
+            }
+            cp_async_wait_all();
+            __syncthreads();
+
+            const int n4 = S.chunk_cnt[ck][0], n3 = S.chunk_cnt[ck][1], n2 = S.chunk_cnt[ck][2],
+                      n1 = S.chunk_cnt[ck][3];
+            int c = c0;
+            for (const int e = c + n4; c < e; ++c) channel_step<G, 4>(S, c, c - c0, blk, l, acc);
+            for (const int e = c + n3; c < e; ++c) channel_step<G, 3>(S, c, c - c0, blk, l, acc);
+            for (const int e = c + n2; c < e; ++c) channel_step<G, 2>(S, c, c - c0, blk, l, acc);
+#pragma unroll 2
+            for (const int e = c + n1; c < e; ++c) channel_step<G, 1>(S, c, c - c0, blk, l, acc);
+        }
+
+        // ---- epilogue.  acc[pr] holds tokens half*32 + l + 8*m of the lane's
+        // block for (half, m) = (pr >> 1, 2*(pr & 1) + e), e = 0 (.x) or 1 (.y).
+        const int64_t tok0 = b0 * kBlockTokens + blk * kBlockTokens + l;
         if (a.mode == kDense) {
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int64_t i = tok_tile0 + local0 + 8 * m;
-                if (i < a.n)
+            for (int pr = 0; pr < 4; ++pr)
 #pragma unroll
-                    for (int g = 0; g < G; ++g) a.scores[(h * G + g) * a.n + i] = acc[s][m][g];
-            }
+                for (int e = 0; e < 2; ++e) {
+                    const int64_t i = tok0 + (pr >> 1) * 32 + 8 * (2 * (pr & 1) + e);
+                    if (i < a.n)
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            a.scores[(h * G + g) * a.n + i] = e ? acc[pr][g].y : acc[pr][g].x;
+                }
         } else if (a.mode == kSample) {
-            const int64_t lt = static_cast<int64_t>(blockIdx.x) * kScanTileTokens;
+            const int64_t lt0 = ltile * kScanTileTokens + blk * kBlockTokens + l;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int64_t i = tok_tile0 + local0 + 8 * m;
+            for (int pr = 0; pr < 4; ++pr)
 #pragma unroll
-                for (int g = 0; g < G; ++g)
-                    a.sample[(h * G + g) * a.n_sample + lt + local0 + 8 * m] = (i < a.n) ? acc[s][m][g] : -INFINITY;
-            }
+                for (int e = 0; e < 2; ++e) {
+                    const int off = (pr >> 1) * 32 + 8 * (2 * (pr & 1) + e);
+                    const bool in = tok0 + off < a.n;
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+                        a.sample[(h * G + g) * a.n_sample + lt0 + off] =
+                            in ? (e ? acc[pr][g].y : acc[pr][g].x) : -INFINITY;
+                }
         } else {
             bool any = false;
 #pragma unroll
-            for (int m = 0; m < 4; ++m)
+            for (int pr = 0; pr < 4; ++pr)
 #pragma unroll
-                for (int g = 0; g < G; ++g)
-                    any |= (tok_tile0 + local0 + 8 * m < a.n) && acc[s][m][g] >= tau_s[g];
+                for (int e = 0; e < 2; ++e) {
+                    const bool in = tok0 + (pr >> 1) * 32 + 8 * (2 * (pr & 1) + e) < a.n;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) any |= in && (e ? acc[pr][g].y : acc[pr][g].x) >= S.tau[g];
+                }
             if (__any_sync(0xffffffffu, any)) {
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int64_t i = tok_tile0 + local0 + 8 * m;
+                for (int pr = 0; pr < 4; ++pr)
 #pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        const bool p = (i < a.n) && acc[s][m][g] >= tau_s[g];
-                        const unsigned mask = __ballot_sync(0xffffffffu, p);
-                        if (mask) {
-                            const int leader = __ffs(mask) - 1;
-                            int base = 0;
-                            if (lane == leader) base = atomicAdd(&a.hdr[h * G + g].count, __popc(mask));
-                            base = __shfl_sync(0xffffffffu, base, leader);
-                            if (p) {
-                                const int64_t pos = base + __popc(mask & ((1u << lane) - 1u));
-                                if (pos < a.cap)
-                                    a.entries[(h * G + g) * a.cap + pos] =
-                                        make_int2(static_cast<int>(i), __float_as_int(acc[s][m][g]));
+                    for (int e = 0; e < 2; ++e) {
+                        const int64_t i = tok0 + (pr >> 1) * 32 + 8 * (2 * (pr & 1) + e);
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            const float sv = e ? acc[pr][g].y : acc[pr][g].x;
+                            const bool p = (i < a.n) && sv >= S.tau[g];
+                            const unsigned mask = __ballot_sync(0xffffffffu, p);
+                            if (mask) {
+                                const int leader = __ffs(mask) - 1;
+                                int base = 0;
+                                if (lane == leader) base = atomicAdd(&a.hdr[h * G + g].count, __popc(mask));
+                                base = __shfl_sync(0xffffffffu, base, leader);
+                                if (p) {
+                                    const int64_t pos = base + __popc(mask & ((1u << lane) - 1u));
+                                    if (pos < a.cap)
+                                        a.entries[(h * G + g) * a.cap + pos] =
+                                            make_int2(static_cast<int>(i), __float_as_int(sv));
+                                }
                             }
                         }
                     }
-                }
             }
         }
     }
 }
 
 template <int G>
-int launch_scan_g(const ScanArgs& a, unsigned tiles, unsigned H, cudaStream_t stream)
+int launch_scan_g(ScanArgs a, int64_t ltiles, unsigned H, cudaStream_t stream)
 {
-    scan_kernel<G><<<dim3(tiles, H), kScanThreads, 0, stream>>>(a);
+    const size_t smem = sizeof(SharedScan<G>);
+    const cudaError_t e = cudaFuncSetAttribute(scan_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_status(e);
+    // Several tiles per CTA amortise the per-CTA plan set-up, as long as the
+    // grid still fills the GPU several times over.
+    int64_t per = ltiles * H / 2400;
+    a.tiles_per_cta = static_cast<int>(per < 1 ? 1 : (per > 8 ? 8 : per));
+    const unsigned gx = static_cast<unsigned>(ceil_div(ltiles, a.tiles_per_cta));
+    scan_kernel<G><<<dim3(gx, H), kScanThreads, smem, stream>>>(a);
     return launch_status();
 }
 
-int launch_scan_mode(const ScanArgs& a, int G, unsigned tiles, unsigned H, cudaStream_t stream)
+int launch_scan_mode(const ScanArgs& a, int G, int64_t ltiles, unsigned H, cudaStream_t stream)
 {
     switch (G) {
-        case 1: return launch_scan_g<1>(a, tiles, H, stream);
-        case 2: return launch_scan_g<2>(a, tiles, H, stream);
-        case 3: return launch_scan_g<3>(a, tiles, H, stream);
-        case 4: return launch_scan_g<4>(a, tiles, H, stream);
-        case 5: return launch_scan_g<5>(a, tiles, H, stream);
-        case 6: return launch_scan_g<6>(a, tiles, H, stream);
-        case 7: return launch_scan_g<7>(a, tiles, H, stream);
-        default: return launch_scan_g<8>(a, tiles, H, stream);
+        case 1: return launch_scan_g<1>(a, ltiles, H, stream);
+        case 2: return launch_scan_g<2>(a, ltiles, H, stream);
+        case 3: return launch_scan_g<3>(a, ltiles, H, stream);
+        case 4: return launch_scan_g<4>(a, ltiles, H, stream);
+        case 5: return launch_scan_g<5>(a, ltiles, H, stream);
+        case 6: return launch_scan_g<6>(a, ltiles, H, stream);
+        case 7: return launch_scan_g<7>(a, ltiles, H, stream);
+        default: return launch_scan_g<8>(a, ltiles, H, stream);
     }
 }
 
@@ -301,7 +440,8 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
     a.active = active;
     a.n_active = n_active;
     a.q = q;
-    const unsigned tiles = static_cast<unsigned>(ceil_div(n, kScanTileTokens));
+    const int64_t tiles = ceil_div(n, kScanTileTokens);
+    a.tiles = tiles;
     if (mode == FATHOM_SCAN_DENSE) {
         a.scores = scores;
         a.mode = kDense;
@@ -319,7 +459,7 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
         if (L.sample_tiles > 0) {
             a.mode = kSample;
             a.tile_stride = L.tile_stride;
-            int st = launch_scan_mode(a, G, static_cast<unsigned>(L.sample_tiles), static_cast<unsigned>(H), stream);
+            int st = launch_scan_mode(a, G, L.sample_tiles, static_cast<unsigned>(H), stream);
             if (st) return st;
         }
         int st = launch_tau(a.sample, a.hdr, L.heads, L.n_sample, L.m_rank, stream);
