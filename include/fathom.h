@@ -27,7 +27,7 @@
  *   - Layout names list dimensions outermost first; all arrays are dense
  *     row-major unless a stride argument says otherwise.
  *   - Limits: 32 <= D <= 256 with D % 32 == 0; 1 <= G <= 8; 1 <= k <= 4096
- *     and G*k <= 16384 for top-k; n < 2^31.
+ *     and G*k <= 16384 for top-k (k <= 1024 on the candidate path); n < 2^31.
  */
 #ifndef FATHOM_H
 #define FATHOM_H
@@ -177,8 +177,10 @@ size_t fathom_scan_cand_bytes(int64_t H, int G, int64_t n, int k);
  * for D <= 128.  No 1/sqrt(D) factor is applied (it does not change ranks).
  *
  *   planes, scales  DEVICE (or mapped page-locked host memory), as written
- *                   by fathom_pack with the same nb_stride.  planes must be
- *                   16-byte aligned and nb_stride even.
+ *                   by fathom_pack with the same nb_stride.  Both must be
+ *                   16-byte aligned and nb_stride a multiple of 8 (as
+ *                   fathom_nb_stride() gives); FATHOM_ERR_UNSUPPORTED
+ *                   otherwise.
  *   active, n_active  DEVICE, from fathom_plan / fathom_plan_fixed.
  *   q               DEVICE, fp32 [H][G][D].
  *   mode            FATHOM_SCAN_DENSE: write scores.

@@ -166,7 +166,7 @@ int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
     if (H == 0 || n == 0) return FATHOM_OK;
     const int64_t nb = ceil_div(n, kBlockTokens);
     if (nb_stride < nb) return FATHOM_ERR_INVALID_ARG;
-    if ((nb_stride & 1) || !aligned(planes, 16) || !aligned(scales, 2) || !aligned(active, 2) ||
+    if ((nb_stride & 7) || !aligned(planes, 16) || !aligned(scales, 16) || !aligned(active, 2) ||
         !aligned(n_active, 4) || !aligned(q, 4))
         return FATHOM_ERR_UNSUPPORTED;
     FATHOM_TRY(check_device_ptr(planes));
@@ -179,7 +179,7 @@ int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
         FATHOM_TRY(check_device_ptr(scores));
     } else {
         if (k < 1 || k > n) return FATHOM_ERR_INVALID_ARG;
-        if (k > kMaxK) return FATHOM_ERR_UNSUPPORTED;
+        if (k > kMaxCandK) return FATHOM_ERR_UNSUPPORTED;
         if (!aligned(cand, 16)) return FATHOM_ERR_UNSUPPORTED;
         FATHOM_TRY(check_device_ptr(cand));
         if (cand_bytes < cand_layout(H, G, n, k).total) return FATHOM_ERR_WORKSPACE;
@@ -210,6 +210,7 @@ int fathom_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
         if (!aligned(scores, 4)) return FATHOM_ERR_UNSUPPORTED;
         FATHOM_TRY(check_device_ptr(scores));
     } else {
+        if (k > kMaxCandK) return FATHOM_ERR_UNSUPPORTED;
         if (!aligned(cand, 16)) return FATHOM_ERR_UNSUPPORTED;
         FATHOM_TRY(check_device_ptr(cand));
     }

@@ -15,6 +15,8 @@ constexpr int kPlanes = 4;         // 4-bit codes
 constexpr int kMaxD = 256;
 constexpr int kMaxG = 8;
 constexpr int kMaxK = 4096;
+constexpr int kMaxCandK = 1024;      // largest k of the candidate path
+constexpr int kCandGather = 8 * kMaxCandK;   // survivors a top-k CTA gathers per head
 constexpr int kMaxUnion = 16384;
 
 // Record a CUDA error for fathom_last_cuda_error() and map it to a status.
@@ -41,12 +43,15 @@ __device__ __forceinline__ float key_to_float(uint32_t k)
 }
 
 // ---------------------------------------------------------------------
-// Candidate buffer of a CANDIDATE scan.  Per (group, head): a header,
-// a sample-score area (only when a threshold is sampled) and `cap`
-// (index, score) entries.
+// Candidate buffer of a CANDIDATE scan, per (group, head):
+//   header (count, tau, sample size);
+//   sample scores (only when a threshold is sampled);
+//   survivors: without a sample, every key at its own index (n entries);
+//   with a sample, a fixed slot of `tslot` entries per scan tile, plus one
+//   count per tile (a count above tslot marks an overflowed slot).
 // ---------------------------------------------------------------------
 struct CandHeader {
-    int32_t count;   // keys that reached tau (may exceed cap: those were dropped)
+    int32_t count;   // without a sample: n; with one: unused (tile counts hold the totals)
     float tau;       // threshold the main pass used
     int32_t n_sample;
     int32_t pad;
@@ -54,12 +59,14 @@ struct CandHeader {
 
 struct CandLayout {
     int64_t heads;        // H * G
-    int64_t cap;          // entries per head
-    int64_t sample_tiles; // tiles in the sample (0: tau = -inf, no sample)
+    int64_t tiles;        // scan tiles of n
+    int64_t tslot;        // survivor slots per (tile, head); 0 without a sample
+    int64_t cap;          // entries per head: n (no sample) or tiles * tslot
+    int64_t sample_tiles; // tiles in the sample (0: tau = -inf, every key kept)
     int64_t tile_stride;  // sample takes every tile_stride-th tile
     int64_t n_sample;     // sample tokens per head (sample_tiles * tile tokens)
     int64_t m_rank;       // tau = m_rank-th largest sample score
-    size_t off_hdr, off_sample, off_entries, total;
+    size_t off_hdr, off_sample, off_counts, off_entries, total;
 };
 
 constexpr int kScanTileBlocks = 16;                       // 1024 tokens per scan tile

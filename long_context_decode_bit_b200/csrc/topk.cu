@@ -113,7 +113,8 @@ __host__ __device__ inline int pow2_at_least(int x)
 // Threshold for the candidate pass: tau = m-th largest sample score of each
 // head (or -inf without a sample); also resets the candidate counters.
 __global__ void __launch_bounds__(kTopkThreads)
-tau_kernel(const float* __restrict__ sample, CandHeader* __restrict__ hdr, int64_t n_sample, int64_t m_rank)
+tau_kernel(const float* __restrict__ sample, CandHeader* __restrict__ hdr, int64_t n_sample, int64_t m_rank,
+           int64_t n_keys)
 {
     __shared__ uint32_t hist[kRadixBins];
     __shared__ uint32_t sh[2];
@@ -126,7 +127,8 @@ tau_kernel(const float* __restrict__ sample, CandHeader* __restrict__ hdr, int64
         tau = key_to_float(r.T);
     }
     if (threadIdx.x == 0) {
-        hdr[hg].count = 0;
+        // Without a sample every key is kept, at its own index (n entries).
+        hdr[hg].count = n_sample > 0 ? 0 : static_cast<int32_t>(n_keys);
         hdr[hg].tau = tau;
         hdr[hg].n_sample = static_cast<int32_t>(n_sample);
         hdr[hg].pad = 0;
@@ -136,8 +138,9 @@ tau_kernel(const float* __restrict__ sample, CandHeader* __restrict__ hdr, int64
 struct TopkArgs {
     const float* scores;        // dense [H*G][n] or null
     const CandHeader* hdr;      // candidate mode
+    const int32_t* tile_counts; // [H*G][tiles] (with a threshold sample)
     const int2* entries;
-    int64_t cap;
+    int64_t cap, tiles, tslot;
     int64_t n;
     int k, kpow2;
     int32_t* idx;               // [H*G][k]
@@ -150,8 +153,9 @@ topk_kernel(const TopkArgs a)
     uint64_t* win = reinterpret_cast<uint64_t*>(smem);                        // kpow2
     int32_t* ties = reinterpret_cast<int32_t*>(win + a.kpow2);               // kMaxTies
     uint32_t* hist = reinterpret_cast<uint32_t*>(ties + kMaxTies);           // kRadixBins
+    int2* gathered = reinterpret_cast<int2*>(hist + kRadixBins);             // kCandGather (tile slots)
     __shared__ uint32_t sh[2];
-    __shared__ int w_cnt, t_cnt, warp_eq[kTopkThreads / 32];
+    __shared__ int w_cnt, t_cnt, warp_eq[kTopkThreads / 32], g_cnt, g_bad;
 
     const int64_t hg = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -164,13 +168,34 @@ topk_kernel(const TopkArgs a)
     if (a.scores) {
         count = a.n;
         sc = a.scores + hg * a.n;
-    } else {
-        count = a.hdr[hg].count;
+    } else if (a.tslot == 0) {
+        count = a.hdr[hg].count;            // every key kept at its own index
         ent = a.entries + hg * a.cap;
-        if (count < k || count > a.cap) {   // could not prove exactness
+        if (count < k || count > a.cap) {
             for (int r = tid; r < k; r += blockDim.x) out[r] = -1;
             return;
         }
+    } else {
+        // Gather the non-empty tile slots into shared memory.
+        if (tid == 0) { g_cnt = 0; g_bad = 0; }
+        __syncthreads();
+        const int32_t* tc = a.tile_counts + hg * a.tiles;
+        const int2* src = a.entries + hg * a.cap;
+        for (int64_t t = tid; t < a.tiles; t += blockDim.x) {
+            const int c = tc[t];
+            if (c <= 0) continue;
+            if (c > a.tslot) { g_bad = 1; continue; }       // slot overflowed: keys were dropped
+            const int base = atomicAdd(&g_cnt, c);
+            if (base + c > kCandGather) { g_bad = 1; continue; }
+            for (int e = 0; e < c; ++e) gathered[base + e] = src[t * a.tslot + e];
+        }
+        __syncthreads();
+        count = g_cnt;
+        if (g_bad || count < k || count > kCandGather) {   // could not prove exactness
+            for (int r = tid; r < k; r += blockDim.x) out[r] = -1;
+            return;
+        }
+        ent = gathered;
     }
     auto key_at = [&](int64_t i) -> uint32_t {
         return sc ? order_key(sc[i]) : order_key(__int_as_float(ent[i].y));
@@ -288,15 +313,16 @@ union_kernel(const int32_t* __restrict__ idx, int G, int k, int upow2, int32_t* 
 }  // namespace
 
 int launch_tau(const float* sample, CandHeader* hdr, int64_t heads, int64_t n_sample, int64_t m_rank,
-               cudaStream_t stream)
+               int64_t n_keys, cudaStream_t stream)
 {
-    tau_kernel<<<static_cast<unsigned>(heads), kTopkThreads, 0, stream>>>(sample, hdr, n_sample, m_rank);
+    tau_kernel<<<static_cast<unsigned>(heads), kTopkThreads, 0, stream>>>(sample, hdr, n_sample, m_rank, n_keys);
     return launch_status();
 }
 
-size_t topk_smem_bytes(int k)
+size_t topk_smem_bytes(int k, bool gather)
 {
-    return sizeof(uint64_t) * pow2_at_least(k) + sizeof(int32_t) * kMaxTies + sizeof(uint32_t) * kRadixBins;
+    return sizeof(uint64_t) * pow2_at_least(k) + sizeof(int32_t) * kMaxTies + sizeof(uint32_t) * kRadixBins +
+           (gather ? sizeof(int2) * kCandGather : 0);
 }
 
 int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
@@ -308,14 +334,19 @@ int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
     a.k = k;
     a.kpow2 = pow2_at_least(k);
     a.idx = idx;
+    bool gather = false;
     if (!scores) {
         const CandLayout L = cand_layout(H, G, n, k);
         const char* base = static_cast<const char*>(cand);
         a.hdr = reinterpret_cast<const CandHeader*>(base + L.off_hdr);
+        a.tile_counts = reinterpret_cast<const int32_t*>(base + L.off_counts);
         a.entries = reinterpret_cast<const int2*>(base + L.off_entries);
         a.cap = L.cap;
+        a.tiles = L.tiles;
+        a.tslot = L.tslot;
+        gather = L.tslot > 0;
     }
-    const size_t smem = topk_smem_bytes(k);
+    const size_t smem = topk_smem_bytes(k, gather);
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_status(e);

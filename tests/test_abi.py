@@ -50,9 +50,10 @@ def test_host_only_entry_points(lib):
     small = lib.fathom_scan_cand_bytes(2, 4, 1000, 64)        # no sample: cap = n
     assert small >= 2 * 4 * (16 + 1000 * 8)
     big = lib.fathom_scan_cand_bytes(288, 4, 2 ** 20, 512)
-    # 1152 heads x (4096 entries of 8 B + 32768 sample scores of 4 B) + headers
-    assert big >= 1152 * (4096 * 8 + 32768 * 4)
-    assert big < 1152 * (4096 * 8 + 32768 * 4) + 1152 * 16 + 4096
+    # 1152 heads x (1024 tiles x 16 survivor slots of 8 B + 1024 tile counts
+    # + 32768 sample scores of 4 B) + headers
+    per_head = 1024 * 16 * 8 + 1024 * 4 + 32768 * 4
+    assert 1152 * per_head <= big < 1152 * (per_head + 16) + 4 * 256
 
 
 def test_rejections_before_any_cuda_call(lib):
