@@ -6,17 +6,18 @@
 // where c_t is the key's t-bit prefix code read from the first t plane rows
 // of channel j.  The K bytes are read once for all G heads.
 //
-// Work layout.  A CTA (4 warps) walks `tiles_per_cta` consecutive tiles of
-// 16 64-token blocks of one group.  Each warp owns 4 blocks of a tile; a
-// lane owns 8 tokens of one block: bit positions l, l+8, l+16, l+24
-// (l = lane & 7) of the block's low and of its high 32-bit plane half.
-//
-// Per tile, the active channels (sorted by depth once per CTA) are staged
-// in chunks: their plane words go to shared memory with cp.async, laid out
-// [block][slot][64-bit word] so that a lane fetches all planes of a channel
-// with one or two 128-bit loads; the coefficients (q_{g,j} 2^-t) * s_{b,j}
-// of every (channel, block) are computed once into shared memory as
-// duplicated pairs for the packed fp32x2 FMA.
+// Work layout.  A CTA is one producer warp and four consumer warps working
+// on one group.  The CTA walks `tiles_per_cta` tiles of 16 64-token blocks;
+// the group's active channels (sorted by depth once per CTA) are split into
+// chunks, and one (tile, chunk) pair is a pipeline unit.
+//   - The producer streams each unit's plane rows (16 words, 128 B per row)
+//     and fp16 scale rows into a 3-stage shared-memory ring with 16-byte
+//     cp.async copies, and hands stages over through named barriers.
+//   - Consumer warp w owns blocks 4w..4w+3 of a tile; a lane owns 8 tokens
+//     of one block: bit positions l, l+8, l+16, l+24 (l = lane & 7) of the
+//     block's low and of its high 32-bit plane half.  Each warp first forms
+//     the coefficients (q_{g,j} 2^-t) * s_{b,j} of its own 4 blocks in a
+//     warp-private table, then decodes and accumulates.
 //
 // Decoding, per channel and per 32-bit half (four tokens at once):
 //   - depth 1: one shift moves each token's sign bit to bit 7 of its own
@@ -25,28 +26,34 @@
 //   - depth t >= 2: one funnel-shift rotation per plane moves plane p's
 //     four bits to bit 7-p of four bytes and one AND/OR merges them, so
 //     byte m holds c_t << (8-t); a byte permute drops it into the low
-//     mantissa of 1.5 * 2^23 and one packed FMA with exact constants gives
-//     the odd integers 2 c_t - 2^t + 1 of two tokens.
-//   - then G packed FMAs per token pair add coefficient * value.
+//     mantissa of 1.5 * 2^23 and one FMA with exact constants gives the odd
+//     integer 2 c_t - 2^t + 1.
+//   - then packed fp32x2 FMAs over pairs of heads add coefficient * value.
 // There are no tensor cores: the contraction is a gathered, variable-depth
 // GEMV whose operand must be decoded bit by bit first.
 //
 // Output modes: DENSE writes every score; SAMPLE writes the scores of a
 // strided subset of tiles to the candidate buffer's sample area; CANDIDATE
-// appends (index, score) of keys whose score reaches the head's threshold
-// with warp-aggregated atomics.
+// keeps keys whose score reaches the head's threshold: at their own index
+// when there is no threshold sample, else in this tile's slot range.
 #include "common.cuh"
 
 namespace fathom {
 
 namespace {
 
-constexpr int kScanThreads = 128;
-constexpr int kScanWarps = kScanThreads / 32;
-constexpr int kBlocksPerWarp = kScanTileBlocks / kScanWarps;  // 4
-constexpr int kChunkCh = 40;        // channels per staging chunk
-constexpr int kChunkSlots = 64;     // 64-bit plane words per block per chunk
-constexpr int kWordStride = kChunkSlots * 8 + 16;  // bytes per staged block (+16 spreads banks)
+constexpr int kConsumerWarps = 4;
+constexpr int kScanThreads = 32 * (kConsumerWarps + 1);         // + one producer warp
+constexpr int kBlocksPerWarp = kScanTileBlocks / kConsumerWarps;  // 4
+constexpr int kStages = 3;   // the stage_sync/stage_arrive helpers spell out 3 stages
+constexpr int kChunkCh = 40;        // channels per chunk
+constexpr int kChunkRows = 64;      // plane rows per chunk
+constexpr int kRowBytes = kScanTileBlocks * 8;   // one plane row of a tile: 128 B
+
+// Named barriers (0 is __syncthreads).
+constexpr int kBarReady = 1;                 // + stage: producer -> consumers
+constexpr int kBarEmpty = 1 + kStages;       // + stage: consumers -> producer
+constexpr int kBarConsumers = 1 + 2 * kStages;
 
 enum ScanMode { kDense = 0, kSample = 1, kCandidate = 2 };
 
@@ -68,44 +75,66 @@ struct ScanArgs {
     int mode;
 };
 
-// Slots a channel of depth t takes in a staged block: depth 3 and 4 an
-// aligned 32-byte quad, depth 2 an aligned 16-byte pair, depth 1 one word.
-// Channels are staged in descending depth, so the alignment holds.
-__host__ __device__ constexpr int slots_of(int t) { return t >= 3 ? 4 : t; }
-
-// Coefficient pairs stored per (channel, block): G rounded up to even, so
-// every record starts on a 16-byte boundary for the 16-byte stores.
+// Heads are handled in pairs for the packed FMA; odd G gets a zero pad.
 template <int G>
-__host__ __device__ constexpr int coef_stride() { return (G + 1) & ~1; }
+__host__ __device__ constexpr int head_pairs() { return (G + 1) / 2; }
+
+// Stored pairs per (channel, block): an even count once there are two or
+// more, so that every record starts on 16 bytes for the 16-byte loads.
+template <int G>
+__host__ __device__ constexpr int coef_pairs() { return head_pairs<G>() == 1 ? 1 : (head_pairs<G>() + 1) & ~1; }
 
 template <int G>
 struct SharedScan {
-    __align__(16) unsigned char words[2][kScanTileBlocks * kWordStride];   // double-buffered planes
-    __align__(16) uint16_t rawscale[2][kChunkCh * kScanTileBlocks];        // double-buffered fp16 scales
-    __align__(16) float2 coef[kChunkCh * kScanTileBlocks * coef_stride<G>()];   // duplicated pairs
-    float qs[kMaxD * G];             // q_{g,j} * 2^-t, depth-sorted order
+    __align__(16) uint64_t words[kStages][kChunkRows * kScanTileBlocks];     // ring: plane rows
+    __align__(16) uint16_t rawscale[kStages][kChunkCh * kScanTileBlocks];    // ring: fp16 scale rows
+    __align__(16) float2 coef[kConsumerWarps][kChunkCh * kBlocksPerWarp * coef_pairs<G>()];
+    float qs[kMaxD * 2 * head_pairs<G>()];   // q_{g,j} * 2^-t, depth-sorted order, zero-padded heads
     uint16_t chan[kMaxD];            // depth-sorted entries j | t << 8
-    uint8_t slot[kMaxD];             // slot of each sorted channel within its chunk
+    uint16_t rowsrc[kMaxD * kPlanes];// plane rows in chunk order: j << 2 | p
     int16_t chunk_begin[kMaxD + 1];  // chunk boundaries in sorted order
+    int16_t chunk_row0[kMaxD + 1];   // first row of each chunk
     int16_t chunk_cnt[kMaxD][4];     // per chunk: channels of depth 4, 3, 2, 1
     int n_chunks;
     float tau[G];
-    int direct[G];                    // no threshold sample: every key is kept, at its own index
-    int tile_cnt[G];                  // survivors of the current tile per head
+    int direct[G];                   // no threshold sample: every key is kept, at its own index
+    int tile_cnt[G];                 // survivors of the current tile per head
 };
 
-__device__ __forceinline__ void cp_async8(void* smem, const void* gmem, bool valid)
+// Named barriers with compile-time ids (a run-time id reserves all 16).
+template <int ID, int COUNT>
+__device__ __forceinline__ void bar_sync()
 {
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    const int n = valid ? 8 : 0;   // 0: zero fill, nothing is read
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+    asm volatile("bar.sync %0, %1;\n" ::"n"(ID), "n"(COUNT) : "memory");
+}
+
+template <int ID, int COUNT>
+__device__ __forceinline__ void bar_arrive()
+{
+    asm volatile("bar.arrive %0, %1;\n" ::"n"(ID), "n"(COUNT) : "memory");
+}
+
+template <int BASE>
+__device__ __forceinline__ void stage_sync(int st)
+{
+    if (st == 0) bar_sync<BASE + 0, kScanThreads>();
+    else if (st == 1) bar_sync<BASE + 1, kScanThreads>();
+    else bar_sync<BASE + 2, kScanThreads>();
+}
+
+template <int BASE>
+__device__ __forceinline__ void stage_arrive(int st)
+{
+    if (st == 0) bar_arrive<BASE + 0, kScanThreads>();
+    else if (st == 1) bar_arrive<BASE + 1, kScanThreads>();
+    else bar_arrive<BASE + 2, kScanThreads>();
 }
 
 // 16-byte copy of which only the first `bytes` (0..16) are read; the rest is zero-filled.
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int bytes)
 {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(bytes) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
@@ -114,18 +143,18 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 // Depth-1 values of the four tokens of one 32-bit half: +-1.0f.
-__device__ __forceinline__ void values_depth1(uint32_t w, int l, float2& v01, float2& v23)
+__device__ __forceinline__ void values_depth1(uint32_t w, int l, float (&v)[4])
 {
     const uint32_t y = ((w << (7 - l)) & 0x80808080u) ^ 0xBFBFBFBFu;
-    v01.x = __uint_as_float(__byte_perm(y, 0x00800000u, 0x0654u));
-    v01.y = __uint_as_float(__byte_perm(y, 0x00800000u, 0x1654u));
-    v23.x = __uint_as_float(__byte_perm(y, 0x00800000u, 0x2654u));
-    v23.y = __uint_as_float(__byte_perm(y, 0x00800000u, 0x3654u));
+    v[0] = __uint_as_float(__byte_perm(y, 0x00800000u, 0x0654u));
+    v[1] = __uint_as_float(__byte_perm(y, 0x00800000u, 0x1654u));
+    v[2] = __uint_as_float(__byte_perm(y, 0x00800000u, 0x2654u));
+    v[3] = __uint_as_float(__byte_perm(y, 0x00800000u, 0x3654u));
 }
 
 // Depth-T (T >= 2) values of four tokens from T plane halves.
 template <int T>
-__device__ __forceinline__ void values_depth(const uint32_t (&w)[4], int l, float2& v01, float2& v23)
+__device__ __forceinline__ void values_depth(const uint32_t (&w)[4], int l, float (&v)[4])
 {
     uint32_t code = 0;
 #pragma unroll
@@ -135,108 +164,152 @@ __device__ __forceinline__ void values_depth(const uint32_t (&w)[4], int l, floa
     }
     constexpr float mul = static_cast<float>(1u << T) / 128.0f;                          // 2^(t-7)
     constexpr float sub = 1.5f * static_cast<float>(1u << (16 + T)) + static_cast<float>((1u << T) - 1);
-    const float2 m2 = make_float2(mul, mul), s2 = make_float2(-sub, -sub);
-    float2 f01, f23;
-    f01.x = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7650u));
-    f01.y = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7651u));
-    f23.x = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7652u));
-    f23.y = __uint_as_float(__byte_perm(code, 0x4B400000u, 0x7653u));
-    v01 = __ffma2_rn(f01, m2, s2);   // exact odd integers
-    v23 = __ffma2_rn(f23, m2, s2);
+#pragma unroll
+    for (int m = 0; m < 4; ++m)   // exact odd integers
+        v[m] = __fmaf_rn(__uint_as_float(__byte_perm(code, 0x4B400000u, 0x7650u + m)), mul, -sub);
 }
 
-// One channel of depth T for the lane's block: 8 tokens (4 pairs) x G heads.
-// wrow: the channel's staged words in the lane's block; cf: its G
-// duplicated coefficient pairs for that block.
+__device__ __forceinline__ uint2 lds_u2(uint32_t addr)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr)
+{
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];\n" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
+// One channel of depth T for the lane's block: 8 tokens x G heads.
+// wrow: shared address of the channel's first plane row at the lane's block
+// column; cf: shared address of its head-pair coefficients for that block.
 template <int G, int T>
-__device__ __forceinline__ void channel_step(const unsigned char* wrow, const float2* cf, int l, float2 (&acc)[4][G])
+__device__ __forceinline__ void channel_step(uint32_t wrow, uint32_t cf, int l, float2 (&acc)[8][head_pairs<G>()])
 {
     uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
-    if (T == 1) {
-        const uint2 x = *reinterpret_cast<const uint2*>(wrow);
-        lo[0] = x.x; hi[0] = x.y;
-    } else {
-        const uint4 x = *reinterpret_cast<const uint4*>(wrow);
-        lo[0] = x.x; hi[0] = x.y; lo[1] = x.z; hi[1] = x.w;
-        if (T >= 3) {
-            const uint4 y = *reinterpret_cast<const uint4*>(wrow + 16);
-            lo[2] = y.x; hi[2] = y.y; lo[3] = y.z; hi[3] = y.w;
-        }
-    }
-    float2 v[4];
-    if (T == 1) {
-        values_depth1(lo[0], l, v[0], v[1]);
-        values_depth1(hi[0], l, v[2], v[3]);
-    } else {
-        values_depth<T>(lo, l, v[0], v[1]);
-        values_depth<T>(hi, l, v[2], v[3]);
-    }
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const float2 k2 = cf[g];
+    for (int p = 0; p < T; ++p) {
+        const uint2 x = lds_u2(wrow + p * kRowBytes);
+        lo[p] = x.x;
+        hi[p] = x.y;
+    }
+    float v[8];
+    if (T == 1) {
+        values_depth1(lo[0], l, *reinterpret_cast<float(*)[4]>(&v[0]));
+        values_depth1(hi[0], l, *reinterpret_cast<float(*)[4]>(&v[4]));
+    } else {
+        values_depth<T>(lo, l, *reinterpret_cast<float(*)[4]>(&v[0]));
+        values_depth<T>(hi, l, *reinterpret_cast<float(*)[4]>(&v[4]));
+    }
+    constexpr int GP = head_pairs<G>();
+    float2 k[GP];
 #pragma unroll
-        for (int pr = 0; pr < 4; ++pr) acc[pr][g] = __ffma2_rn(v[pr], k2, acc[pr][g]);
+    for (int gp = 0; gp + 1 < GP; gp += 2) {
+        const float4 k4 = lds_f4(cf + gp * 8);
+        k[gp] = make_float2(k4.x, k4.y);
+        k[gp + 1] = make_float2(k4.z, k4.w);
+    }
+    if (GP & 1) k[GP - 1] = lds_f2(cf + (GP - 1) * 8);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const float2 vv = make_float2(v[m], v[m]);
+#pragma unroll
+        for (int gp = 0; gp < GP; ++gp) acc[m][gp] = __ffma2_rn(vv, k[gp], acc[m][gp]);
     }
 }
 
-// All channels of one depth class of a chunk.
 template <int G, int T>
-__device__ __forceinline__ void depth_class(const unsigned char* wrow, const float2* cf, int count, int l,
-                                            float2 (&acc)[4][G])
+__device__ __forceinline__ void depth_class(uint32_t& wrow, uint32_t& cf, int count, int l,
+                                            float2 (&acc)[8][head_pairs<G>()])
 {
     for (int i = 0; i < count; ++i) {
         channel_step<G, T>(wrow, cf, l, acc);
-        wrow += slots_of(T) * 8;
-        cf += kScanTileBlocks * coef_stride<G>();
+        wrow += T * kRowBytes;
+        cf += kBlocksPerWarp * coef_pairs<G>() * 8;
     }
 }
 
 template <int G>
-__global__ void __launch_bounds__(kScanThreads, 4)
+__device__ __forceinline__ float acc_at(const float2 (&acc)[8][head_pairs<G>()], int m, int g)
+{
+    return (g & 1) ? acc[m][g >> 1].y : acc[m][g >> 1].x;
+}
+
+#ifndef FATHOM_SCAN_MIN_CTAS
+#define FATHOM_SCAN_MIN_CTAS 3
+#endif
+#ifndef FATHOM_SCAN_TILES_CAP
+#define FATHOM_SCAN_TILES_CAP 32
+#endif
+
+template <int G>
+__global__ void __launch_bounds__(kScanThreads, FATHOM_SCAN_MIN_CTAS)
 scan_kernel(const ScanArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SharedScan<G>& S = *reinterpret_cast<SharedScan<G>*>(smem_raw);
+    constexpr int GP = head_pairs<G>();
 
     const int64_t h = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int D = a.D;
     const int na = min(max(a.n_active[h], 0), D);   // trust nothing beyond D entries
 
-    // ---- the group's plan, sorted by depth (4, 3, 2, 1), ascending j within a depth
-    if (tid < 32) {
+    // ---- the group's plan: one parallel read of the active list, then a
+    // sort by depth (4, 3, 2, 1), ascending j within a depth
+    for (int i = tid; i < na; i += kScanThreads) {
+        const uint16_t e = a.active[h * D + i];
+        const int j = e & 0xFF;
+        int tt = min(e >> 8, kPlanes);
+        if (j >= D) tt = 0;       // malformed entry: read nothing
+        S.rowsrc[i] = static_cast<uint16_t>(j | (tt << 8));   // staging area until the sort is done
+    }
+    __syncthreads();
+    if (warp == 0) {
         int base = 0;
         for (int t = 4; t >= 1; --t) {
             for (int i0 = 0; i0 < na; i0 += 32) {
                 const int i = i0 + lane;
                 int j = 0, tt = 0;
                 if (i < na) {
-                    const uint16_t e = a.active[h * D + i];
+                    const uint16_t e = S.rowsrc[i];
                     j = e & 0xFF;
-                    tt = min(e >> 8, kPlanes);
-                    if (j >= D) tt = 0;       // malformed entry: read nothing
+                    tt = e >> 8;
                 }
                 const unsigned bal = __ballot_sync(0xffffffffu, tt == t);
                 if (tt == t) S.chan[base + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(j | (t << 8));
                 base += __popc(bal);
             }
         }
-        __syncwarp();
-        // Chunks of at most kChunkCh channels and kChunkSlots staged words.
+        __syncwarp();   // every lane has read its entries before lane 0 rewrites rowsrc
+        // Chunks of at most kChunkCh channels and kChunkRows plane rows, and
+        // the row list (j, p) of every chunk in order.
         if (lane == 0) {
-            int c = 0, k = 0;
+            int c = 0, k = 0, row = 0;
             while (c < base) {
                 S.chunk_begin[k] = static_cast<int16_t>(c);
-                int n4 = 0, n3 = 0, n2 = 0, n1 = 0, slots = 0, ch = 0;
+                S.chunk_row0[k] = static_cast<int16_t>(row);
+                int n4 = 0, n3 = 0, n2 = 0, n1 = 0, rows = 0, ch = 0;
                 while (c < base && ch < kChunkCh) {
-                    const int t = S.chan[c] >> 8;
-                    if (slots + slots_of(t) > kChunkSlots) break;
-                    S.slot[c] = static_cast<uint8_t>(slots);
-                    slots += slots_of(t);
+                    const int j = S.chan[c] & 0xFF, t = S.chan[c] >> 8;
+                    if (rows + t > kChunkRows) break;
+                    for (int p = 0; p < t; ++p) S.rowsrc[row + rows + p] = static_cast<uint16_t>((j << 2) | p);
+                    rows += t;
                     n4 += t == 4; n3 += t == 3; n2 += t == 2; n1 += t == 1;
                     ch++;
                     c++;
                 }
+                row += rows;
                 S.chunk_cnt[k][0] = static_cast<int16_t>(n4);
                 S.chunk_cnt[k][1] = static_cast<int16_t>(n3);
                 S.chunk_cnt[k][2] = static_cast<int16_t>(n2);
@@ -245,10 +318,12 @@ scan_kernel(const ScanArgs a)
             }
             if (k == 0) {   // no active channel: one empty chunk, every score is 0
                 S.chunk_begin[0] = 0;
+                S.chunk_row0[0] = 0;
                 S.chunk_cnt[0][0] = S.chunk_cnt[0][1] = S.chunk_cnt[0][2] = S.chunk_cnt[0][3] = 0;
                 k = 1;
             }
             S.chunk_begin[k] = static_cast<int16_t>(c);
+            S.chunk_row0[k] = static_cast<int16_t>(row);
             S.n_chunks = k;
         }
     }
@@ -259,17 +334,15 @@ scan_kernel(const ScanArgs a)
         const int j = S.chan[i] & 0xFF, t = S.chan[i] >> 8;
         const float sc = __uint_as_float(static_cast<uint32_t>(127 - t) << 23);  // 2^-t
 #pragma unroll
-        for (int g = 0; g < G; ++g) S.qs[i * G + g] = __fmul_rn(a.q[(h * G + g) * D + j], sc);
+        for (int g = 0; g < 2 * GP; ++g)
+            S.qs[i * 2 * GP + g] = g < G ? __fmul_rn(a.q[(h * G + g) * D + j], sc) : 0.0f;
     }
     if (a.mode == kCandidate && tid < G) {
         S.tau[tid] = a.hdr[h * G + tid].tau;
         S.direct[tid] = a.hdr[h * G + tid].n_sample == 0;
         S.tile_cnt[tid] = 0;
     }
-    __syncthreads();   // qs and tau visible to every warp, even with no chunk to stage
-
-    const int l = lane & 7;
-    const int blk = warp * kBlocksPerWarp + (lane >> 3);   // the lane's block within a tile
+    __syncthreads();   // plan, coefficients' q part and thresholds visible to every warp
 
     // Tiles of this CTA that exist.
     int64_t tiles_here = a.tiles_per_cta;
@@ -280,149 +353,145 @@ scan_kernel(const ScanArgs a)
     }
     const int units = static_cast<int>(tiles_here) * n_chunks;
 
-    // Stage unit u = (tile, chunk) into buffer `buf`: plane words (8-byte
-    // copies, zero-filled past the last block) and raw fp16 scales.
-    auto issue = [&](int u, int buf) {
-        const int ti = u / n_chunks, ck = u % n_chunks;
-        const int64_t ltile = static_cast<int64_t>(blockIdx.x) * a.tiles_per_cta + ti;
-        const int64_t b0 = ltile * a.tile_stride * kScanTileBlocks;
-        const int c0 = S.chunk_begin[ck], c1 = S.chunk_begin[ck + 1];
-        {
-            const int b = tid & 15;
-            const int64_t blkg = b0 + b;
-            const bool valid = blkg < a.nb;
-            for (int c = c0 + (tid >> 4); c < c1; c += kScanThreads / 16) {
-                const int j = S.chan[c] & 0xFF, t = S.chan[c] >> 8;
-                const uint64_t* src = a.planes + (h * D + j) * kPlanes * a.nb_stride + (valid ? blkg : 0);
-                unsigned char* dst = S.words[buf] + b * kWordStride + S.slot[c] * 8;
-                for (int p = 0; p < t; ++p) cp_async8(dst + p * 8, src + p * a.nb_stride, valid);
+    if (warp == kConsumerWarps) {
+        // ================= producer warp =================
+        for (int u = 0; u < units; ++u) {
+            const int st = u % kStages;
+            if (u >= kStages) stage_sync<kBarEmpty>(st);   // consumers freed this stage
+            const int ti = u / n_chunks, ck = u % n_chunks;
+            const int64_t ltile = static_cast<int64_t>(blockIdx.x) * a.tiles_per_cta + ti;
+            const int64_t b0 = ltile * a.tile_stride * kScanTileBlocks;
+            const int64_t valid_blocks = a.nb - b0;   // >= 1
+            const int r0 = S.chunk_row0[ck], rows = S.chunk_row0[ck + 1] - r0;
+            const int c0 = S.chunk_begin[ck], nc = S.chunk_begin[ck + 1] - c0;
+            // Plane rows: 8 pieces of 16 B (2 blocks each) per row.
+            for (int idx = lane; idx < rows * 8; idx += 32) {
+                const int r = idx >> 3, part = idx & 7;
+                const int src_rc = S.rowsrc[r0 + r];
+                const int64_t row = (h * D + (src_rc >> 2)) * kPlanes + (src_rc & 3);
+                const int64_t vb = valid_blocks - 2 * part;
+                const int bytes = vb >= 2 ? 16 : (vb == 1 ? 8 : 0);
+                const uint64_t* src = a.planes + row * a.nb_stride + (bytes ? b0 + 2 * part : 0);
+                cp_async16(&S.words[st][r * kScanTileBlocks + 2 * part], src, bytes);
+            }
+            // Scale rows: 2 pieces of 16 B (8 blocks each) per channel.
+            for (int idx = lane; idx < nc * 2; idx += 32) {
+                const int c = idx >> 1, part = idx & 1;
+                const int j = S.chan[c0 + c] & 0xFF;
+                const int64_t vb = valid_blocks - 8 * part;
+                const int bytes = vb >= 8 ? 16 : (vb > 0 ? static_cast<int>(vb) * 2 : 0);
+                const uint16_t* src = a.scales + (h * D + j) * a.nb_stride + (bytes ? b0 + 8 * part : 0);
+                cp_async16(&S.rawscale[st][c * kScanTileBlocks + 8 * part], src, bytes);
+            }
+            cp_async_commit();
+            if (u >= 1) {
+                cp_async_wait<1>();   // unit u-1 has landed
+                stage_arrive<kBarReady>((u - 1) % kStages);
             }
         }
-        // Scales: two 16-byte copies (8 blocks each) per channel.
-        for (int idx = tid; idx < (c1 - c0) * 2; idx += kScanThreads) {
-            const int cl = idx >> 1, part = idx & 1;
-            const int j = S.chan[c0 + cl] & 0xFF;
-            const int64_t first = b0 + part * 8;
-            const int64_t nvalid = a.nb - first;
-            const int bytes = nvalid >= 8 ? 16 : (nvalid > 0 ? static_cast<int>(nvalid) * 2 : 0);
-            const uint16_t* src = a.scales + (h * D + j) * a.nb_stride + (bytes > 0 ? first : 0);
-            cp_async16(S.rawscale[buf] + cl * kScanTileBlocks + part * 8, src, bytes);
-        }
-        cp_async_commit();
-    };
-
-    float2 acc[4][G];
-    if (units > 0) issue(0, 0);
-    for (int u = 0; u < units; ++u) {
-        const int buf = u & 1;
-        const int ti = u / n_chunks, ck = u % n_chunks;
-        if (u + 1 < units) {
-            issue(u + 1, buf ^ 1);
-            cp_async_wait<1>();
-        } else {
+        if (units >= 1) {
             cp_async_wait<0>();
+            stage_arrive<kBarReady>((units - 1) % kStages);
         }
-        __syncthreads();   // unit u's words and scales are in place
+        return;
+    }
 
-        const int c0 = S.chunk_begin[ck], c1 = S.chunk_begin[ck + 1];
-        // Coefficients of every (channel, block) as duplicated pairs: each
-        // thread writes one 16-byte pair of pairs, consecutive threads
-        // consecutive 16 bytes.
-        constexpr int kPairs = (G + 1) / 2;
-        for (int idx = tid; idx < (c1 - c0) * kScanTileBlocks * kPairs; idx += kScanThreads) {
-            const int gp = idx % kPairs, cb = idx / kPairs;
-            const int cl = cb / kScanTileBlocks, b = cb % kScanTileBlocks;
-            const float s = __half2float(__ushort_as_half(S.rawscale[buf][cl * kScanTileBlocks + b]));
-            const float* qsc = S.qs + (c0 + cl) * G;
-            float2* dst = S.coef + cb * coef_stride<G>() + 2 * gp;
-            const float v0 = __fmul_rn(qsc[2 * gp], s);
-            if (2 * gp + 1 < G) {
-                const float v1 = __fmul_rn(qsc[2 * gp + 1], s);
-                *reinterpret_cast<float4*>(dst) = make_float4(v0, v0, v1, v1);
-            } else {
-                *dst = make_float2(v0, v0);
-            }
+    // ================= consumer warps =================
+    const int l = lane & 7;
+    const int bl = lane >> 3;                      // block of the lane within the warp's 4
+    const int blk = warp * kBlocksPerWarp + bl;    // block of the lane within the tile
+    float2* wcoef = S.coef[warp];
+
+    float2 acc[8][GP];
+    for (int u = 0; u < units; ++u) {
+        const int st = u % kStages;
+        const int ti = u / n_chunks, ck = u % n_chunks;
+        stage_sync<kBarReady>(st);   // unit u is in stage st
+
+        const int c0 = S.chunk_begin[ck], nc = S.chunk_begin[ck + 1] - c0;
+        // Coefficients of the warp's 4 blocks: (channel, block) -> G/2 head pairs.
+        for (int idx = lane; idx < nc * kBlocksPerWarp; idx += 32) {
+            const int c = idx >> 2, b = idx & 3;
+            const float s = __half2float(__ushort_as_half(S.rawscale[st][c * kScanTileBlocks + warp * kBlocksPerWarp + b]));
+            const float* q2 = S.qs + (c0 + c) * 2 * GP;
+            float2* dst = wcoef + (c * kBlocksPerWarp + b) * coef_pairs<G>();
+#pragma unroll
+            for (int gp = 0; gp < GP; ++gp) dst[gp] = make_float2(__fmul_rn(q2[2 * gp], s), __fmul_rn(q2[2 * gp + 1], s));
         }
-        __syncthreads();
+        __syncwarp();
 
         if (ck == 0) {
 #pragma unroll
-            for (int pr = 0; pr < 4; ++pr)
+            for (int m = 0; m < 8; ++m)
 #pragma unroll
-                for (int g = 0; g < G; ++g) acc[pr][g] = make_float2(0.0f, 0.0f);
+                for (int gp = 0; gp < GP; ++gp) acc[m][gp] = make_float2(0.0f, 0.0f);
         }
         {
             const int n4 = S.chunk_cnt[ck][0], n3 = S.chunk_cnt[ck][1], n2 = S.chunk_cnt[ck][2],
                       n1 = S.chunk_cnt[ck][3];
-            const unsigned char* wrow = S.words[buf] + blk * kWordStride;   // slots start at 0 per chunk
-            constexpr int cs = coef_stride<G>();
-            const float2* cf = S.coef + blk * cs;
+            uint32_t wrow = static_cast<uint32_t>(__cvta_generic_to_shared(&S.words[st][blk]));  // row 0, lane's block
+            uint32_t cf = static_cast<uint32_t>(__cvta_generic_to_shared(wcoef + bl * coef_pairs<G>()));
             depth_class<G, 4>(wrow, cf, n4, l, acc);
-            wrow += n4 * 32; cf += n4 * kScanTileBlocks * cs;
             depth_class<G, 3>(wrow, cf, n3, l, acc);
-            wrow += n3 * 32; cf += n3 * kScanTileBlocks * cs;
             depth_class<G, 2>(wrow, cf, n2, l, acc);
-            wrow += n2 * 16; cf += n2 * kScanTileBlocks * cs;
             depth_class<G, 1>(wrow, cf, n1, l, acc);
         }
+        __syncwarp();   // the warp's coefficient table may be rebuilt after this
 
         if (ck == n_chunks - 1) {
-            // ---- epilogue.  acc[pr] holds tokens half*32 + l + 8*m of the lane's
-            // block for (half, m) = (pr >> 1, 2*(pr & 1) + e), e = 0 (.x) or 1 (.y).
+            // ---- epilogue: token m of the lane is blk*64 + (m >> 2)*32 + l + 8*(m & 3).
             const int64_t ltile = static_cast<int64_t>(blockIdx.x) * a.tiles_per_cta + ti;
             const int64_t b0 = ltile * a.tile_stride * kScanTileBlocks;
             const int64_t tok0 = b0 * kBlockTokens + blk * kBlockTokens + l;
             if (a.mode == kDense) {
 #pragma unroll
-                for (int pr = 0; pr < 4; ++pr)
+                for (int m = 0; m < 8; ++m) {
+                    const int64_t i = tok0 + (m >> 2) * 32 + 8 * (m & 3);
+                    if (i < a.n)
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int64_t i = tok0 + (pr >> 1) * 32 + 8 * (2 * (pr & 1) + e);
-                        if (i < a.n)
-#pragma unroll
-                            for (int g = 0; g < G; ++g)
-                                a.scores[(h * G + g) * a.n + i] = e ? acc[pr][g].y : acc[pr][g].x;
-                    }
+                        for (int g = 0; g < G; ++g) a.scores[(h * G + g) * a.n + i] = acc_at<G>(acc, m, g);
+                }
             } else if (a.mode == kSample) {
                 const int64_t lt0 = ltile * kScanTileTokens + blk * kBlockTokens + l;
 #pragma unroll
-                for (int pr = 0; pr < 4; ++pr)
+                for (int m = 0; m < 8; ++m) {
+                    const int off = (m >> 2) * 32 + 8 * (m & 3);
+                    const bool in = tok0 + off < a.n;
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int off = (pr >> 1) * 32 + 8 * (2 * (pr & 1) + e);
-                        const bool in = tok0 + off < a.n;
-#pragma unroll
-                        for (int g = 0; g < G; ++g)
-                            a.sample[(h * G + g) * a.n_sample + lt0 + off] =
-                                in ? (e ? acc[pr][g].y : acc[pr][g].x) : -INFINITY;
-                    }
+                    for (int g = 0; g < G; ++g)
+                        a.sample[(h * G + g) * a.n_sample + lt0 + off] = in ? acc_at<G>(acc, m, g) : -INFINITY;
+                }
             } else {
-                // Candidates.  Without a threshold sample every key is kept at
-                // its own index.  Otherwise survivors go to this tile's fixed
-                // slot range (position from a shared counter, no global
-                // atomic); the tile's count is written once all warps are done.
                 const int64_t ptile = ltile * a.tile_stride;
+                // Most lanes hold no survivor: test each head's maximum first.
+                bool any = false;
 #pragma unroll
-                for (int pr = 0; pr < 4; ++pr)
+                for (int g = 0; g < G; ++g) {
+                    float mx = acc_at<G>(acc, 0, g);
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int64_t i = tok0 + (pr >> 1) * 32 + 8 * (2 * (pr & 1) + e);
+                    for (int m = 1; m < 8; ++m) mx = fmaxf(mx, acc_at<G>(acc, m, g));
+                    any |= mx >= S.tau[g];
+                }
+                if (any)
 #pragma unroll
-                        for (int g = 0; g < G; ++g) {
-                            const float sv = e ? acc[pr][g].y : acc[pr][g].x;
-                            if (i < a.n && sv >= S.tau[g]) {
-                                const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
-                                if (S.direct[g]) {
-                                    a.entries[(h * G + g) * a.cap + i] = ent;
-                                } else {
-                                    const int p = atomicAdd(&S.tile_cnt[g], 1);
-                                    if (p < a.tslot) a.entries[(h * G + g) * a.cap + ptile * a.tslot + p] = ent;
-                                }
+                for (int m = 0; m < 8; ++m) {
+                    const int64_t i = tok0 + (m >> 2) * 32 + 8 * (m & 3);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float sv = acc_at<G>(acc, m, g);
+                        if (i < a.n && sv >= S.tau[g]) {
+                            const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
+                            if (S.direct[g]) {
+                                a.entries[(h * G + g) * a.cap + i] = ent;
+                            } else {
+                                const int p = atomicAdd(&S.tile_cnt[g], 1);
+                                if (p < a.tslot) a.entries[(h * G + g) * a.cap + ptile * a.tslot + p] = ent;
                             }
                         }
                     }
+                }
                 if (a.tslot > 0) {
-                    __syncthreads();
+                    bar_sync<kBarConsumers, 32 * kConsumerWarps>();   // every consumer warp has appended
                     if (tid < G) {
                         a.tile_counts[(h * G + tid) * a.tiles + ptile] = S.tile_cnt[tid];
                         S.tile_cnt[tid] = 0;
@@ -430,9 +499,8 @@ scan_kernel(const ScanArgs a)
                 }
             }
         }
-        __syncthreads();   // buffers of unit u may be refilled from here on
+        if (u + kStages < units) stage_arrive<kBarEmpty>(st);   // stage st may be refilled
     }
-
 }
 
 template <int G>
@@ -444,8 +512,8 @@ int launch_scan_g(ScanArgs a, int64_t ltiles, unsigned H, cudaStream_t stream)
     if (e != cudaSuccess) return cuda_status(e);
     // Several tiles per CTA amortise the per-CTA plan set-up, as long as the
     // grid still fills the GPU several times over.
-    int64_t per = ltiles * H / 2400;
-    a.tiles_per_cta = static_cast<int>(per < 1 ? 1 : (per > 8 ? 8 : per));
+    int64_t per = ltiles * H / 1800;
+    a.tiles_per_cta = static_cast<int>(per < 1 ? 1 : (per > FATHOM_SCAN_TILES_CAP ? FATHOM_SCAN_TILES_CAP : per));
     const unsigned gx = static_cast<unsigned>(ceil_div(ltiles, a.tiles_per_cta));
     scan_kernel<G><<<dim3(gx, H), kScanThreads, smem, stream>>>(a);
     return launch_status();
