@@ -1,0 +1,104 @@
+"""Parity at the benchmark's full sizes, in the launch configuration the
+benchmark times (all groups of the step in one batched launch, candidate
+path), on outputs the oracle can compute one by one:
+
+- the plan of every group, bit-exact;
+- planes and scales of sampled groups, bit-exact;
+- the scores of sampled keys of sampled groups, within 1e-5 of their L1 scale;
+- the top-k and union of sampled groups against the oracle's full sort.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bench
+from long_context_decode_bit_b200 import fathom, inputs
+from _util import SCORE_RTOL, assert_topk_sets_match, keys_for_oracle, np_u16, np_u64
+
+pytestmark = pytest.mark.gpu
+
+SAMPLED_GROUPS = (0, 157)   # first group, and one from the middle layers
+
+
+@pytest.fixture(scope="module")
+def step_1m():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fathom.load()
+    w = inputs.STEP_1M
+    dev = torch.device("cuda", 0)
+    planes, scales, s2, q, _ = bench.build_index(w, dev)
+    st = fathom.Step(planes, scales, w.n, s2, w.G, w.k, budget=48)
+    idx, uni, cnt = st.run(q)
+    torch.cuda.synchronize()
+    yield w, planes, scales, s2, q, st
+    del planes, scales
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("h", SAMPLED_GROUPS)
+def test_fullsize_step_matches_oracle_on_sampled_group(step_1m, orc, h):
+    w, planes, scales, s2, q, st = step_1m
+    # planes/scales of group h from its own keys, regenerated (same seed)
+    k = inputs.keys(w, h, h + 1, device="cuda")
+    p_ref, s_ref = orc.pack(keys_for_oracle(k), nb_stride=planes.shape[-1])
+    del k
+    assert np.array_equal(np_u64(planes[h:h + 1]), p_ref)
+    assert np.array_equal(np_u16(scales[h:h + 1]), s_ref)
+    qn = q[h:h + 1].cpu().numpy()
+    d_ref = orc.plan(s2[h:h + 1].cpu().numpy(), qn, 48)[0]
+    depth = st.plan_out[0]
+    assert np.array_equal(depth[h:h + 1].cpu().numpy(), d_ref)
+    # scores of sampled keys (GPU dense scan of this group vs the oracle)
+    ref, l1 = orc.scan(p_ref, s_ref, d_ref, qn, w.n)
+    _, active, na, _ = st.plan_out
+    dense = fathom.scan(planes[h:h + 1], scales[h:h + 1], w.n, active[h:h + 1], na[h:h + 1], q[h:h + 1])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(h)
+    sample = np.concatenate([rng.integers(0, w.n, 20000), np.arange(0, 2048), np.arange(w.n - 2048, w.n)])
+    g_sc = dense.cpu().numpy()[0][:, sample].astype(np.float64)
+    err = np.abs(g_sc - ref[0][:, sample])
+    assert np.all(err <= SCORE_RTOL * l1[0][:, sample])
+    # top-k of the batched candidate step vs the oracle's full sort
+    idx, uni, cnt = st.topk_out
+    r_idx, r_uni, r_cnt = orc.topk(ref, w.k)
+    g_idx = idx[h:h + 1].cpu().numpy()
+    assert int(cnt[h]) > 0
+    assert_topk_sets_match(g_idx, r_idx, ref, l1, w.k)
+    # and exactly the top-k of the GPU's own dense scores of this group
+    g_all = dense.cpu().numpy()[0]
+    for g in range(w.G):
+        want = np.lexsort((np.arange(w.n), -g_all[g].astype(np.float64)))[:w.k]
+        assert np.array_equal(g_idx[0, g], want)
+    u = np.unique(g_idx.reshape(-1))
+    assert int(cnt[h]) == len(u) and np.array_equal(uni[h, :len(u)].cpu().numpy(), u)
+
+
+def test_fullsize_plan_every_group_bit_exact(step_1m, orc):
+    w, planes, scales, s2, q, st = step_1m
+    depth, active, na, theta = st.plan_out
+    d_ref, a_ref, na_ref, _ = orc.plan(s2.cpu().numpy(), q.cpu().numpy(), 48)
+    assert np.array_equal(depth.cpu().numpy(), d_ref)
+    assert np.array_equal(np_u16(active), a_ref)
+    assert np.array_equal(na.cpu().numpy(), na_ref)
+    assert int(torch.min(st.topk_out[2])) > 0   # no group needed the dense rerun
+
+
+def test_step_128k_sampled_groups(orc):
+    """The 288 x 131072 step (a second full-size configuration)."""
+    w = inputs.STEP_128K
+    dev = torch.device("cuda", 0)
+    planes, scales, s2, q, _ = bench.build_index(w, dev)
+    st = fathom.Step(planes, scales, w.n, s2, w.G, w.k, budget=48)
+    idx, uni, cnt = st.run(q)
+    torch.cuda.synchronize()
+    d_ref = orc.plan(s2.cpu().numpy(), q.cpu().numpy(), 48)[0]
+    assert np.array_equal(st.plan_out[0].cpu().numpy(), d_ref)
+    for h in (5, 287):
+        k = inputs.keys(w, h, h + 1, device="cuda")
+        p_ref, s_ref = orc.pack(keys_for_oracle(k), nb_stride=planes.shape[-1])
+        assert np.array_equal(np_u64(planes[h:h + 1]), p_ref)
+        qn = q[h:h + 1].cpu().numpy()
+        ref, l1 = orc.scan(p_ref, s_ref, d_ref[h:h + 1], qn, w.n)
+        r_idx = orc.topk(ref, w.k)[0]
+        assert_topk_sets_match(idx[h:h + 1].cpu().numpy(), r_idx, ref, l1, w.k)
