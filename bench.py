@@ -53,6 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-sweep", action="store_true", help="skip the budget / per-layer sweep")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--cpu-groups", type=int, default=1, help="groups in the CPU-oracle sample")
+    ap.add_argument("--host-resident", action="store_true",
+                    help="index in page-locked host memory, read over the host link (multi-session case)")
+    ap.add_argument("--sessions", type=int, default=3, help="sessions of the host-resident case")
     ap.add_argument("--quiet", action="store_true")
     return ap.parse_args(argv)
 
@@ -372,6 +375,76 @@ def run_gpu(args):
     return result if rank == 0 else None
 
 
+def h2d_bandwidth(device, nbytes=1 << 30, reps=10):
+    """Best-of-10 pinned host -> device copy bandwidth (GB/s): the link roofline."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize(device)
+        best = max(best, nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    return best
+
+
+def run_host_resident(args):
+    """Multi-session decode step with every session's index in page-locked
+    host memory, scanned zero-copy over the host link.  The pages' case is 16
+    sessions of 256k..1M tokens (about 205 GB); the session count is scaled to
+    the host's memory and reported."""
+    import torch
+    from long_context_decode_bit_b200 import fathom, inputs
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    log = (lambda *a: print(*a, file=sys.stderr, flush=True)) if not args.quiet else (lambda *a: None)
+    fathom.load()
+    lens = inputs.session_lengths(args.sessions, 262144, 1048576, seed=4242)
+    sessions = []
+    t0 = time.time()
+    for si, n in enumerate(lens):
+        w = inputs.Workload(f"session{si}", H=288, n=n, seed=500 + si)
+        planes, scales, s2, q, _ = build_index(w, device, log=log)
+        hp = torch.empty(planes.shape, dtype=planes.dtype, pin_memory=True)
+        hs = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+        hp.copy_(planes)
+        hs.copy_(scales)
+        del planes, scales
+        torch.cuda.empty_cache()
+        sessions.append((w, hp, hs, s2, q))
+    host_gb = sum(x[1].numel() * 8 + x[2].numel() * 2 for x in sessions) / 1e9
+    log(f"[bench] {len(lens)} host-resident sessions {lens} ({host_gb:.1f} GB pinned) in {time.time() - t0:.0f}s")
+    link = h2d_bandwidth(device)
+    out = {}
+    for name, kw in (("B48", dict(budget=48)), ("fixed136_r32", dict(fixed_r=32))):
+        steps = [fathom.Step(hp, hs, w.n, s2, w.G, w.k, **kw) for (w, hp, hs, s2, q) in sessions]
+
+        def one(ev):
+            for st, (w, hp, hs, s2, q) in zip(steps, sessions):
+                st.run(q, check_overflow=False)
+        one(None)
+        torch.cuda.synchronize(device)
+        fb = sum(st.repair(q) for st, (w, _, _, _, q) in zip(steps, sessions))
+        alg = sum(plan_bytes(st, w)[0] for st, (w, *_) in zip(steps, sessions))
+        tot, _ = time_steps(one, args.steps, args.warmup, device)
+        ms = tot / args.steps
+        keys = sum(w.H * w.n for (w, *_) in sessions)
+        out[name] = {"ms_per_step": ms, "keys_per_s": keys / (ms / 1e3), "alg_bytes": alg,
+                     "link_GBps": alg / (ms / 1e3) / 1e9, "link_frac": alg / (ms / 1e3) / 1e9 / link,
+                     "fallback_groups": fb}
+        del steps
+    return {"metric": "host-resident multi-session step: keys scanned/s and host-link GB/s vs measured H2D roofline",
+            "value": out["B48"]["keys_per_s"], "unit": "keys/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "host-resident sessions, Qwen3-8B shape (288 groups, D=128, G=4, k=512)",
+                       "sessions": len(lens), "lengths": lens, "pinned_GB": host_gb,
+                       "scaled_from": "16 sessions (about 205 GB) to fit the host's memory"},
+            "link_roofline": {"h2d_GBps_best_of_10": link}, "budgets": out}
+
+
 def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     """Step time at other budgets, the fixed 136-bit scan on the same data,
     and the layer-sequential launch pattern (36 x 8 groups)."""
@@ -484,7 +557,12 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
-    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if args.impl == "reference":
+        res = run_reference(args)
+    elif args.host_resident:
+        res = run_host_resident(args)
+    else:
+        res = run_gpu(args)
     if res is not None:
         print(json.dumps(res), flush=True)
 
