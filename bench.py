@@ -163,6 +163,18 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def alu_roofline(fmas: int, ms: float, clocks: dict, props) -> dict:
+    """The scan's binding roofline: its fp32 multiply-adds (G per key per
+    active channel) against the FMA pipe, 128 lanes per SM per cycle at the
+    SM clock sampled during the timed region."""
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    peak = props.multi_processor_count * 128 * mhz * 1e6 / 1e12
+    achieved = fmas / (ms / 1e3) / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFMA/s", "frac": achieved / peak,
+            "what": "fp32 FMA pipe: SMs x 128 lanes x sampled SM clock; work = n x G x active channels",
+            "fmas_per_launch": fmas}
+
+
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for name in ("scan.cu", "common.cuh"):
@@ -189,20 +201,26 @@ def profiled_traffic(workload: str, budget: int):
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
-def build_index(w, device, chunk: int = 8, log=print):
+def build_index(w, device, chunk: int = 8, log=print, rotated: bool = False):
     """Generate keys per chunk of groups and pack them at once (the raw keys
-    of the full workload would not fit).  Returns planes, scales, sigma2, q
-    and the pack timing of the first chunk."""
+    of the full workload would not fit).  With ``rotated``, keys and
+    queries are first expressed in each group's calibration eigenbasis.
+    Returns planes, scales, sigma2, q and the pack timing of the first chunk."""
     import torch
-    from long_context_decode_bit_b200 import fathom, inputs
+    from long_context_decode_bit_b200 import basis, fathom, inputs
     nbs = fathom.nb_stride(w.n)
     planes = torch.zeros((w.H, w.D, 4, nbs), dtype=torch.int64, device=device)
     scales = torch.zeros((w.H, w.D, nbs), dtype=torch.int16, device=device)
     sigma2 = torch.empty((w.H, w.D), dtype=torch.float32, device=device)
+    q = inputs.queries(w, 0, w.H, device=device).float().contiguous()
     pack_ms = None
     for h0 in range(0, w.H, chunk):
         h1 = min(w.H, h0 + chunk)
         keys = inputs.keys(w, h0, h1, device=device)
+        if rotated:
+            U = basis.klt_basis(keys[:, :w.n_cal], q[h0:h1])
+            keys = basis.rotate(keys, U)
+            q[h0:h1] = basis.rotate(q[h0:h1], U)
         sigma2[h0:h1] = inputs.calibration_sigma2(keys, w.n_cal)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -212,7 +230,6 @@ def build_index(w, device, chunk: int = 8, log=print):
             torch.cuda.synchronize()
             pack_ms = (e0.elapsed_time(e1), h1 - h0, keys.numel() * keys.element_size())
         del keys
-    q = inputs.queries(w, 0, w.H, device=device).float().contiguous()
     torch.cuda.synchronize()
     ms, groups, kbytes = pack_ms
     out_bytes = groups * w.D * (4 * 8 + 2) * w.nb
@@ -300,6 +317,7 @@ def run_gpu(args):
             step.repair(q)
 
     alg_bytes, bits, na = plan_bytes(step, w)
+    alg_fmas = w.n * w.G * sum(na)   # one fp32 multiply-add per (key, query head, active channel)
     props = torch.cuda.get_device_properties(device)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
     with ClockSampler(gpu_id) as clk:
@@ -357,6 +375,7 @@ def run_gpu(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "kernel": "scan_kernel<4> (FILTER)",
                      "peak_source": f"{peak_src} hbm_gbs (copy)"},
+        "alu_roofline": alu_roofline(alg_fmas, filt_mean, clocks, props),
         "scan": {"ms": filt_mean, "GBps": achieved, "alg_bytes": alg_bytes,
                  "read_bits_per_token": alg_bytes * 8 / (w.H * w.n),
                  "plane_bits_mean": statistics.fmean(bits), "active_channels_mean": statistics.fmean(na),
@@ -474,6 +493,39 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
                      "read_bits_per_token": alg * 8 / (w.H * w.n), "plane_bits_mean": statistics.fmean(bits),
                      "active_channels_mean": statistics.fmean(na), "fallback_groups": fb}
         del st
+    # The rotated-basis run on the Llama-3.1-8B shape (32 layers x 8 KV heads).
+    from long_context_decode_bit_b200 import inputs as _inputs
+    wl = _inputs.STEP_1M_LLAMA if w.n == _inputs.STEP_1M.n else dataclasses.replace(_inputs.STEP_1M_LLAMA, n=w.n)
+    del_planes = None
+    try:
+        rp, rs, rs2, rq, _ = build_index(wl, device, rotated=True)
+        for bname, bb in (("rotated_llama_B48", 48), ("rotated_llama_B136", 136)):
+            st = fathom.Step(rp, rs, wl.n, rs2, wl.G, k, budget=bb)
+
+            def one(ev, st=st):
+                st.run_plan(rq)
+                st.run_prepare(rq)
+                if ev is not None:
+                    ev[0].record()
+                st.run_filter(rq)
+                if ev is not None:
+                    ev[1].record()
+                st.run_topk()
+            one(None)
+            torch.cuda.synchronize(device)
+            fb = st.repair(rq)
+            alg, bits, na = plan_bytes(st, wl)
+            tot, fk = time_steps(one, 5, 2, device, kernel_events=True)
+            fm = statistics.fmean(fk)
+            out[bname] = {"workload": wl.name, "ms_per_step": tot / 5, "scan_ms": fm,
+                          "scan_GBps": alg / (fm / 1e3) / 1e9, "keys_per_s": wl.H * wl.n / (tot / 5 / 1e3),
+                          "read_bits_per_token": alg * 8 / (wl.H * wl.n), "active_channels_mean": statistics.fmean(na),
+                          "fallback_groups": fb}
+            del st
+        del rp, rs
+        torch.cuda.empty_cache()
+    except torch.cuda.OutOfMemoryError:
+        out["rotated_llama"] = "skipped: not enough device memory"
     layers = w.H // 8 if w.H % 8 == 0 else 1
     per = w.H // layers
     steps = [fathom.Step(planes[l * per:(l + 1) * per], scales[l * per:(l + 1) * per], w.n,

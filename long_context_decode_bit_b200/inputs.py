@@ -36,6 +36,10 @@ class Workload:
                  (flat channel scales, as under QK-norm); bf16 queries
                  N(0, 1) with 8..12 dominant channels per group at 5x,
                  shared by the group's query heads.
+    ``"corr"``   bf16 keys without QK-norm: z ~ N(0, I) mixed by a random
+                 rotation and a decaying spectrum (per group), so channel
+                 variances are uneven and channels correlated; queries as
+                 for ``qknorm``.
     """
     name: str
     H: int
@@ -58,7 +62,8 @@ TINY = Workload("tiny-1x4096-gauss", H=1, n=4096, kind="gauss", n_cal=1024, budg
 LAYER_32K = Workload("qwen3-8b-layer-8x32768", H=8, n=32768, budgets=(48, 68, 92, 136), k=512, seed=1)
 STEP_128K = Workload("qwen3-8b-step-288x131072", H=288, n=131072, budgets=(48,), k=512, seed=2)
 STEP_1M = Workload("qwen3-8b-step-288x1048576", H=288, n=1048576, budgets=(48, 92, 136), k=512, seed=3)
-STEP_1M_LLAMA = Workload("llama3.1-8b-step-256x1048576", H=256, n=1048576, budgets=(48, 92, 136), k=512, seed=4)
+STEP_1M_LLAMA = Workload("llama3.1-8b-step-256x1048576", H=256, n=1048576, kind="corr", budgets=(48, 92, 136),
+                         k=512, seed=4)
 
 WORKLOADS = {w.name: w for w in (TINY, LAYER_32K, STEP_128K, STEP_1M, STEP_1M_LLAMA)}
 
@@ -91,6 +96,13 @@ def keys(w: Workload, h0: int, h1: int, device="cpu") -> torch.Tensor:
             z = torch.randn(n, w.D, generator=g, device=device)
             rms = torch.sqrt(torch.mean(z * z, dim=1, keepdim=True))
             out.append((z / rms).to(torch.bfloat16))
+        elif w.kind == "corr":
+            g = _gen(device, _group_seed(w, h, 0))
+            rot, _ = torch.linalg.qr(torch.randn(w.D, w.D, generator=g, device=device))
+            spectrum = torch.exp(-torch.arange(w.D, device=device, dtype=torch.float32) / 24.0)
+            mix = rot * torch.sqrt(spectrum)[None, :]
+            z = torch.randn(n, w.D, generator=g, device=device)
+            out.append((z @ mix.T).to(torch.bfloat16))
         else:
             raise ValueError(w.kind)
     return torch.stack(out, 0)
@@ -103,7 +115,7 @@ def queries(w: Workload, h0: int, h1: int, device="cpu") -> torch.Tensor:
     for h in range(h0, h1):
         g = _gen(device, _group_seed(w, h, 1))
         q = torch.randn(w.G, w.D, generator=g, device=device)
-        if w.kind == "qknorm":
+        if w.kind in ("qknorm", "corr"):
             m = int(torch.randint(8, 13, (1,), generator=g, device=device).item())
             dom = torch.randperm(w.D, generator=g, device=device)[:m]
             q[:, dom] *= 5.0

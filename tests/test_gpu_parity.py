@@ -205,3 +205,27 @@ def test_candidate_overflow_is_flagged_and_repaired(fathom_gpu, orc):
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy()[1, 3], np.arange(w.k))
     assert torch.all(cnt == w.k)
+
+
+def test_rotated_basis_full_path(fathom_gpu, orc):
+    """Llama-shaped keys (no QK-norm) stored in the rotated basis: the scan
+    sees fp32 rotated keys and queries; parity holds as for any input."""
+    from long_context_decode_bit_b200 import basis
+    w = dataclasses.replace(inputs.STEP_1M_LLAMA, H=3, n=20000, seed=61)
+    k = inputs.keys(w, 0, w.H, device=DEV)
+    q = inputs.queries(w, 0, w.H, device=DEV).float().contiguous()
+    U = basis.klt_basis(k[:, :w.n_cal], q)
+    kr, qr = basis.rotate(k, U), basis.rotate(q, U)
+    s2 = inputs.calibration_sigma2(kr, w.n_cal).contiguous()
+    planes, scales = fathom_gpu.pack(kr)
+    depth, active, na, _ = fathom_gpu.plan(s2, qr, 48)
+    sc = fathom_gpu.scan(planes, scales, w.n, active, na, qr)
+    idx, uni, cnt = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, budget=48).run(qr)
+    torch.cuda.synchronize()
+    p_ref, s_ref = oracle_pack(orc, kr, planes.shape[-1])
+    assert np.array_equal(np_u64(planes), p_ref) and np.array_equal(np_u16(scales), s_ref)
+    d_ref = orc.plan(s2.cpu().numpy(), qr.cpu().numpy(), 48)[0]
+    assert np.array_equal(depth.cpu().numpy(), d_ref)
+    ref, l1 = orc.scan(p_ref, s_ref, d_ref, qr.cpu().numpy(), w.n)
+    assert_scores_close(sc.cpu().numpy(), ref, l1)
+    assert_topk_sets_match(idx.cpu().numpy(), orc.topk(ref, w.k)[0], ref, l1, w.k)
