@@ -470,7 +470,10 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     import torch
     from long_context_decode_bit_b200 import fathom
     out = {}
-    variants = [(f"B{b}", dict(budget=b)) for b in (48, 68, 92, 136)] + [("fixed136_r32", dict(fixed_r=32))]
+    variants = [(f"B{b}", dict(budget=b)) for b in (48, 68, 92, 136)] + [
+        ("fixed136_r32", dict(fixed_r=32)),                        # 32 channels x 4 bits + scales
+        ("sparq68_r16", dict(fixed_r=16)),                         # 16 channels x 4 bits + scales
+        ("thumbnail_2bit", dict(fixed_r=w.D, fixed_bits=2))]       # 2 bits of every channel
     for name, kw in variants:
         st = fathom.Step(planes, scales, w.n, sigma2, w.G, k, **kw)
 

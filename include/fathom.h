@@ -145,15 +145,17 @@ int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D,
                 fathom_stream_t stream);
 
 /*
- * fathom_plan_fixed -- the fixed-depth comparator plan: the r channels with
+ * fathom_plan_fixed -- a fixed-depth comparator plan: the r channels with
  * the largest a_j = |q_{0,j}| + |q_{1,j}| + ... + |q_{G-1,j}| (single
- * precision, that order; ties to the lower j) at depth 4, the others at 0.
- * With r = 32 this is the 136-bit scan of the byte accounting
- * (先算一笔字节账, third bullet: 32 coordinates x 4 bits + a block scale).
- * The group's heads share the channel set so the K bytes are read once.
- * Outputs as fathom_plan.  0 <= r <= D.
+ * precision, that order; ties to the lower j) read at `bits` planes, the
+ * others at 0.  The group's heads share the channel set so the K bytes are
+ * read once.  The comparators of the pages (先算一笔字节账 and 固定深度的浪费在哪):
+ *   r = 32, bits = 4: the 136-bit scan (32 coordinates x 4 bits + scales);
+ *   r = 16, bits = 4: SparQ's 68-bit read;
+ *   r = D,  bits = 2: the thumbnail scan (2 bits of every channel).
+ * Outputs as fathom_plan.  0 <= r <= D, 1 <= bits <= 4.
  */
-int fathom_plan_fixed(const float* q, int64_t H, int G, int D, int r,
+int fathom_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits,
                       uint8_t* depth, uint16_t* active, int32_t* n_active,
                       fathom_stream_t stream);
 

@@ -10,7 +10,7 @@ int launch_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, in
 int launch_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,
                 int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
                 cudaStream_t stream);
-int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, uint8_t* depth, uint16_t* active,
+int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits, uint8_t* depth, uint16_t* active,
                       int32_t* n_active, cudaStream_t stream);
 int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
                 const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
@@ -135,19 +135,19 @@ int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D, co
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
-int fathom_plan_fixed(const float* q, int64_t H, int G, int D, int r, uint8_t* depth, uint16_t* active,
+int fathom_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits, uint8_t* depth, uint16_t* active,
                       int32_t* n_active, fathom_stream_t stream)
 {
     if (H < 0 || H > 0x7FFFFFFF) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
-    if (r < 0 || r > D) return FATHOM_ERR_INVALID_ARG;
+    if (r < 0 || r > D || bits < 1 || bits > kPlanes) return FATHOM_ERR_INVALID_ARG;
     if (H == 0) return FATHOM_OK;
     if (!aligned(q, 4) || !aligned(active, 2) || !aligned(n_active, 4)) return FATHOM_ERR_UNSUPPORTED;
     FATHOM_TRY(check_device_ptr(q));
     FATHOM_TRY(check_device_ptr(depth));
     FATHOM_TRY(check_device_ptr(active));
     FATHOM_TRY(check_device_ptr(n_active));
-    return launch_plan_fixed(q, H, G, D, r, depth, active, n_active, reinterpret_cast<cudaStream_t>(stream));
+    return launch_plan_fixed(q, H, G, D, r, bits, depth, active, n_active, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fathom_scan_cand_bytes(int64_t H, int G, int64_t n, int k)

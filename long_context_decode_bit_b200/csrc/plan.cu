@@ -122,7 +122,7 @@ __global__ void plan_kernel(const float* __restrict__ sigma2, const float* __res
     write_active(j, t, D, h, active, n_active, warp_cnt);
 }
 
-__global__ void plan_fixed_kernel(const float* __restrict__ q, int G, int D, int r,
+__global__ void plan_fixed_kernel(const float* __restrict__ q, int G, int D, int r, int bits,
                                   uint8_t* __restrict__ depth, uint16_t* __restrict__ active,
                                   int32_t* __restrict__ n_active)
 {
@@ -140,7 +140,7 @@ __global__ void plan_fixed_kernel(const float* __restrict__ q, int G, int D, int
         const float b = a_s[i];
         rank += (b > a) || (b == a && i < j);
     }
-    const int t = rank < r ? 4 : 0;
+    const int t = rank < r ? bits : 0;
     depth[h * D + j] = static_cast<uint8_t>(t);
     write_active(j, t, D, h, active, n_active, warp_cnt);
 }
@@ -156,10 +156,10 @@ int launch_plan(const float* sigma2, const float* q, int64_t H, int G, int D, co
     return launch_status();
 }
 
-int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, uint8_t* depth, uint16_t* active,
+int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits, uint8_t* depth, uint16_t* active,
                       int32_t* n_active, cudaStream_t stream)
 {
-    plan_fixed_kernel<<<static_cast<unsigned>(H), D, 0, stream>>>(q, G, D, r, depth, active, n_active);
+    plan_fixed_kernel<<<static_cast<unsigned>(H), D, 0, stream>>>(q, G, D, r, bits, depth, active, n_active);
     return launch_status();
 }
 

@@ -69,7 +69,7 @@ def load(path: str = LIB_PATH):
         "fathom_nb_stride": (I64, [I64]),
         "fathom_pack": (I, [P, I, I64, I64, I, I64, I64, P, P, I64, P]),
         "fathom_plan": (I, [P, P, I64, I, I, P, ctypes.c_int32, P, P, P, P, P]),
-        "fathom_plan_fixed": (I, [P, I64, I, I, I, P, P, P, P]),
+        "fathom_plan_fixed": (I, [P, I64, I, I, I, I, P, P, P, P]),
         "fathom_scan_cand_bytes": (SZ, [I64, I, I64, I]),
         "fathom_scan": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, SZ, I, P]),
         "fathom_topk_workspace_bytes": (SZ, [I64, I, I64, I]),
@@ -151,14 +151,17 @@ def plan(sigma2: torch.Tensor, q: torch.Tensor, budget, out=None, stream=None):
     return depth, active, n_active, theta
 
 
-def plan_fixed(q: torch.Tensor, r: int, out=None, stream=None):
+def plan_fixed(q: torch.Tensor, r: int, out=None, stream=None, bits: int = 4):
+    """Fixed-depth comparator plan: the r channels with the largest
+    sum_g |q| read at ``bits`` planes."""
     H, G, D = q.shape
     dev = q.device
     if out is None:
         out = (torch.empty((H, D), dtype=torch.uint8, device=dev), torch.empty((H, D), dtype=torch.int16, device=dev),
                torch.empty(H, dtype=torch.int32, device=dev))
     depth, active, n_active = out
-    _check(lib().fathom_plan_fixed(_p(q), H, G, D, int(r), _p(depth), _p(active), _p(n_active), _stream(stream)),
+    _check(lib().fathom_plan_fixed(_p(q), H, G, D, int(r), int(bits), _p(depth), _p(active), _p(n_active),
+                                   _stream(stream)),
            "fathom_plan_fixed")
     return depth, active, n_active
 
@@ -225,12 +228,14 @@ class Step:
     candidate pass could not prove its top-k exact.  Buffers are allocated
     once; ``run`` launches only library kernels."""
 
-    def __init__(self, planes, scales, n: int, sigma2, G: int, k: int, budget=48, fixed_r: int | None = None):
+    def __init__(self, planes, scales, n: int, sigma2, G: int, k: int, budget=48, fixed_r: int | None = None,
+                 fixed_bits: int = 4):
         self.planes, self.scales, self.n, self.sigma2, self.k = planes, scales, n, sigma2, k
         self.H, self.D = sigma2.shape
         self.G = G
         self.budget = budget
         self.fixed_r = fixed_r
+        self.fixed_bits = fixed_bits
         dev = sigma2.device
         H, D = self.H, self.D
         self.plan_out = (torch.empty((H, D), dtype=torch.uint8, device=dev),
@@ -247,7 +252,7 @@ class Step:
         if self.fixed_r is None:
             plan(self.sigma2, q, self.budget, out=self.plan_out)
         else:
-            plan_fixed(q, self.fixed_r, out=self.plan_out[:3])
+            plan_fixed(q, self.fixed_r, out=self.plan_out[:3], bits=self.fixed_bits)
         return self.plan_out
 
     def run_prepare(self, q):

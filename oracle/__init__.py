@@ -43,7 +43,7 @@ def _lib():
         lib.orc_plan.restype = I
         lib.orc_plan.argtypes = [P, P, I64, I, I, P, P, P, P, P, P]
         lib.orc_plan_fixed.restype = I
-        lib.orc_plan_fixed.argtypes = [P, I64, I, I, I, P, P, P]
+        lib.orc_plan_fixed.argtypes = [P, I64, I, I, I, I, P, P, P]
         lib.orc_scan.restype = I
         lib.orc_scan.argtypes = [P, P, I64, I, I64, I64, P, P, I, P, P]
         lib.orc_topk.restype = I
@@ -130,14 +130,14 @@ def plan(sigma2: np.ndarray, q: np.ndarray, budget):
     return depth, active, n_active, theta
 
 
-def plan_fixed(q: np.ndarray, r: int):
-    """Fixed-depth plan: the r channels with the largest sum_g |q| at depth 4."""
+def plan_fixed(q: np.ndarray, r: int, bits: int = 4):
+    """Fixed-depth plan: the r channels with the largest sum_g |q| at ``bits`` planes."""
     q = np.ascontiguousarray(q, dtype=np.float32)
     H, G, D = q.shape
     depth = np.zeros((H, D), dtype=np.uint8)
     active = np.zeros((H, D), dtype=np.uint16)
     n_active = np.zeros(H, dtype=np.int32)
-    _check(_lib().orc_plan_fixed(_ptr(q), H, G, D, int(r), _ptr(depth), _ptr(active),
+    _check(_lib().orc_plan_fixed(_ptr(q), H, G, D, int(r), int(bits), _ptr(depth), _ptr(active),
                                  _ptr(n_active)), "plan_fixed")
     return depth, active, n_active
 

@@ -240,8 +240,8 @@ int orc_plan(const float* sigma2, const float* q, int64_t H, int G, int D,
 
 /* Fixed-depth comparator plan: the r channels with the largest         */
 /* sum_g |q_{g,j}| (single precision, fixed order; ties to the lower j) */
-/* are read at all four planes -- the 32-channel, 4-bit scan whose cost */
-/* the byte-accounting section puts at 136 bits per token.              */
+/* are read at `bits` planes -- with r = 32 and 4 planes, the 32-channel */
+/* 4-bit scan the byte-accounting section puts at 136 bits per token.   */
 typedef struct { float a; int j; } orc_rank_t;
 
 static int cmp_rank(const void* x, const void* y)
@@ -253,10 +253,10 @@ static int cmp_rank(const void* x, const void* y)
     return (u->j > v->j) - (u->j < v->j);
 }
 
-int orc_plan_fixed(const float* q, int64_t H, int G, int D, int r,
+int orc_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits,
                    uint8_t* depth, uint16_t* active, int32_t* n_active)
 {
-    if (!q || !depth || H < 0 || G <= 0 || D <= 0 || r < 0 || r > D) return ORC_EINVAL;
+    if (!q || !depth || H < 0 || G <= 0 || D <= 0 || r < 0 || r > D || bits < 1 || bits > 4) return ORC_EINVAL;
     orc_rank_t* rk = (orc_rank_t*)malloc(sizeof(orc_rank_t) * (size_t)D);
     if (!rk) return ORC_ENOMEM;
     for (int64_t h = 0; h < H; ++h) {
@@ -268,10 +268,10 @@ int orc_plan_fixed(const float* q, int64_t H, int G, int D, int r,
         }
         qsort(rk, (size_t)D, sizeof(orc_rank_t), cmp_rank);
         for (int j = 0; j < D; ++j) depth[h * D + j] = 0;
-        for (int i = 0; i < r; ++i) depth[h * D + rk[i].j] = 4;
+        for (int i = 0; i < r; ++i) depth[h * D + rk[i].j] = (uint8_t)bits;
         int na = 0;
         for (int j = 0; j < D; ++j)
-            if (depth[h * D + j] && active) active[h * D + na++] = (uint16_t)(j | (4 << 8));
+            if (depth[h * D + j] && active) active[h * D + na++] = (uint16_t)(j | (bits << 8));
             else if (depth[h * D + j]) na++;
         if (active)
             for (int j = na; j < D; ++j) active[h * D + j] = 0;

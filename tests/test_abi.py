@@ -65,7 +65,9 @@ def test_rejections_before_any_cuda_call(lib):
     assert lib.fathom_plan(n, n, 4, 9, 128, n, 48, n, n, n, n, n) == fathom.ERR_UNSUPPORTED
     assert lib.fathom_plan(n, n, 4, 4, 128, n, 513, n, n, n, n, n) == fathom.ERR_INVALID_ARG
     assert lib.fathom_plan(n, n, 4, 4, 128, n, -1, n, n, n, n, n) == fathom.ERR_INVALID_ARG
-    assert lib.fathom_plan_fixed(n, 4, 4, 128, 129, n, n, n, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_plan_fixed(n, 4, 4, 128, 129, 4, n, n, n, n) == fathom.ERR_INVALID_ARG   # r > D
+    assert lib.fathom_plan_fixed(n, 4, 4, 128, 32, 0, n, n, n, n) == fathom.ERR_INVALID_ARG    # bits = 0
+    assert lib.fathom_plan_fixed(n, 4, 4, 128, 32, 5, n, n, n, n) == fathom.ERR_INVALID_ARG    # bits > 4
     assert lib.fathom_scan(n, n, 1, 128, 100, 2, n, n, n, 4, 5, n, n, 0, 1, n) == fathom.ERR_INVALID_ARG
     assert lib.fathom_scan(n, n, 1, 100, 100, 2, n, n, n, 4, 0, n, n, 0, 1, n) == fathom.ERR_UNSUPPORTED
     assert lib.fathom_topk(n, n, 1, 4, 100, 5, n, n, n, n, 0, n) == fathom.ERR_INVALID_ARG   # neither input

@@ -96,26 +96,26 @@ def test_plan_per_group_budgets_and_edge_importances(fathom_gpu, orc):
     assert np.array_equal(na.cpu().numpy(), na_ref)
 
 
-@pytest.mark.parametrize("r", [0, 1, 16, 32, 128])
-def test_plan_fixed_bit_exact(fathom_gpu, orc, r):
+@pytest.mark.parametrize("r,bits", [(0, 4), (1, 4), (16, 4), (32, 4), (128, 4), (128, 2), (40, 1), (32, 3)])
+def test_plan_fixed_bit_exact(fathom_gpu, orc, r, bits):
     w = dataclasses.replace(inputs.LAYER_32K, H=16, n=4096, seed=22)
     _, q, _ = make(w)
     q[3, :, 7] = q[3, :, 9]  # a tie, broken towards the lower channel
-    depth, active, na = fathom_gpu.plan_fixed(q, r)
+    depth, active, na = fathom_gpu.plan_fixed(q, r, bits=bits)
     torch.cuda.synchronize()
-    d_ref, a_ref, na_ref = orc.plan_fixed(q.cpu().numpy(), r)
+    d_ref, a_ref, na_ref = orc.plan_fixed(q.cpu().numpy(), r, bits)
     assert np.array_equal(depth.cpu().numpy(), d_ref)
     assert np.array_equal(np_u16(active), a_ref)
     assert np.array_equal(na.cpu().numpy(), na_ref)
 
 
-def _full_path(fathom_gpu, orc, w, budget, fixed_r=None):
+def _full_path(fathom_gpu, orc, w, budget, fixed_r=None, fixed_bits=4):
     k, q, s2 = make(w)
     planes, scales = fathom_gpu.pack(k)
     if fixed_r is None:
         depth, active, na, _ = fathom_gpu.plan(s2, q, budget)
     else:
-        depth, active, na = fathom_gpu.plan_fixed(q, fixed_r)
+        depth, active, na = fathom_gpu.plan_fixed(q, fixed_r, bits=fixed_bits)
     sc = fathom_gpu.scan(planes, scales, w.n, active, na, q)
     idx, uni, cnt = fathom_gpu.topk(w.H, w.G, w.n, w.k, scores=sc)
     torch.cuda.synchronize()
@@ -125,7 +125,7 @@ def _full_path(fathom_gpu, orc, w, budget, fixed_r=None):
     if fixed_r is None:
         d_ref = orc.plan(s2.cpu().numpy(), qn, budget)[0]
     else:
-        d_ref = orc.plan_fixed(qn, fixed_r)[0]
+        d_ref = orc.plan_fixed(qn, fixed_r, fixed_bits)[0]
     assert np.array_equal(depth.cpu().numpy(), d_ref)
     ref, l1 = orc.scan(p_ref, s_ref, d_ref, qn, w.n)
     gsc = sc.cpu().numpy()
@@ -156,8 +156,9 @@ def test_layer_32k_full_path(fathom_gpu, orc, budget):
     _full_path(fathom_gpu, orc, inputs.LAYER_32K, budget)
 
 
-def test_layer_32k_fixed_136_bit_scan(fathom_gpu, orc):
-    _full_path(fathom_gpu, orc, inputs.LAYER_32K, None, fixed_r=32)
+@pytest.mark.parametrize("r,bits", [(32, 4), (16, 4), (128, 2)], ids=["136-bit", "sparq-r16", "thumbnail"])
+def test_layer_32k_fixed_depth_comparators(fathom_gpu, orc, r, bits):
+    _full_path(fathom_gpu, orc, inputs.LAYER_32K, None, fixed_r=r, fixed_bits=bits)
 
 
 @pytest.mark.parametrize("n,k", [(1, 1), (37, 37), (64, 5), (5037, 1), (5037, 100)])

@@ -312,17 +312,19 @@ def test_plan_fixed_reduces_to_a_sort(orc):
     H, G, D = 4, 4, 128
     q = rng.standard_normal((H, G, D)).astype(np.float32)
     q[1, :, 5] = q[1, :, 9]  # a tie, broken towards the lower channel
-    for r in (0, 1, 16, 32, 128):
-        depth, active, na = orc.plan_fixed(q, r)
+    for r, bits in ((0, 4), (1, 4), (16, 4), (32, 4), (128, 4), (128, 2), (40, 1), (32, 3)):
+        depth, active, na = orc.plan_fixed(q, r, bits)
         for h in range(H):
             a = np.abs(q[h, 0])
             for g in range(1, G):
                 a = (a + np.abs(q[h, g])).astype(np.float32)
             top = np.lexsort((np.arange(D), -a.astype(np.float64)))[:r]
             want = np.zeros(D, np.uint8)
-            want[top] = 4
+            want[top] = bits
             assert np.array_equal(depth[h], want)
             assert na[h] == r
+            js = np.sort(top)
+            assert np.array_equal(active[h, :r], (js | (bits << 8)).astype(np.uint16))
 
 
 # --------------------------------------------------------------------------
