@@ -245,6 +245,29 @@ int fathom_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
                 void* workspace, size_t ws_bytes, fathom_stream_t stream);
 
 /*
+ * fathom_dequant_rows -- rebuild whole key rows from the index: for group h
+ * and list entry r < row_count[h] (all M entries when row_count is NULL),
+ * token i = rows[h*M + r] and every channel j,
+ *   out[(h*M + r)*D + j] = s_{i/64,j} * (2 c_t - 2^t + 1) / 2^t,  t = bits,
+ * the t-plane prefix value of the stored code (t = 4: the full 4-bit key).
+ * This is how the keys of a KV head's winners can be served from the
+ * channel-major planes themselves (边界, storage-overhead paragraph: the
+ * pages leave this path unbuilt and note a single token is costly to gather
+ * from the channel-major layout).  Values are exact in fp32.  Entries with
+ * i outside [0, n) and rows past row_count give 0.
+ *
+ *   planes, scales  as for fathom_scan (device or mapped host memory).
+ *   rows            DEVICE, int32 [H][M] token indices (e.g. the union of
+ *                   fathom_topk, ascending, which keeps the reads local).
+ *   row_count       DEVICE (may be NULL), int32 [H]; negative counts read as 0.
+ *   bits            1..4.
+ *   out             DEVICE out, fp32 [H][M][D].
+ */
+int fathom_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n,
+                        int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count,
+                        int bits, float* out, fathom_stream_t stream);
+
+/*
  * fathom_scan_topk_noalloc -- fathom_scan in CANDIDATE mode followed by
  * fathom_topk, for callers that cannot allocate device memory.  (The paper
  * has no counterpart: this is a deployment convenience of this library.)

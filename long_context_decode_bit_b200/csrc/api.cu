@@ -18,6 +18,10 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
 int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
                 int32_t* union_idx, int32_t* union_count, cudaStream_t stream);
 
+int launch_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n,
+                        int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count, int bits,
+                        float* out, cudaStream_t stream);
+
 static thread_local int g_last_cuda_error = 0;
 
 int cuda_status(cudaError_t e)
@@ -219,6 +223,27 @@ int fathom_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
     FATHOM_TRY(check_device_ptr(union_count));
     return launch_topk(scores, cand, H, G, n, k, idx, union_idx, union_count,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fathom_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n,
+                        int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count, int bits,
+                        float* out, fathom_stream_t stream)
+{
+    if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31) || M < 0 || M > (1LL << 24)) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
+    if (bits < 1 || bits > kPlanes) return FATHOM_ERR_INVALID_ARG;
+    if (H == 0 || M == 0) return FATHOM_OK;
+    if (nb_stride < ceil_div(n, kBlockTokens)) return FATHOM_ERR_INVALID_ARG;
+    if (!aligned(planes, 8) || !aligned(scales, 2) || !aligned(rows, 4) || !aligned(out, 4) ||
+        (row_count && !aligned(row_count, 4)))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(planes));
+    FATHOM_TRY(check_device_ptr(scales));
+    FATHOM_TRY(check_device_ptr(rows));
+    FATHOM_TRY(check_device_ptr(out));
+    if (row_count) FATHOM_TRY(check_device_ptr(row_count));
+    return launch_dequant_rows(planes, scales, H, D, n, nb_stride, rows, M, row_count, bits, out,
+                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

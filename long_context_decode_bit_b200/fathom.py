@@ -35,7 +35,7 @@ SCAN_FILTER = 3
 EXPORTS = (
     "fathom_version", "fathom_status_string", "fathom_last_cuda_error", "fathom_nb_stride",
     "fathom_pack", "fathom_plan", "fathom_plan_fixed", "fathom_scan_cand_bytes", "fathom_scan",
-    "fathom_topk_workspace_bytes", "fathom_topk", "fathom_scan_topk_noalloc",
+    "fathom_topk_workspace_bytes", "fathom_topk", "fathom_dequant_rows", "fathom_scan_topk_noalloc",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -74,6 +74,7 @@ def load(path: str = LIB_PATH):
         "fathom_scan": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, SZ, I, P]),
         "fathom_topk_workspace_bytes": (SZ, [I64, I, I64, I]),
         "fathom_topk": (I, [P, P, I64, I, I64, I, P, P, P, P, SZ, P]),
+        "fathom_dequant_rows": (I, [P, P, I64, I, I64, I64, P, I64, P, I, P, P]),
         "fathom_scan_topk_noalloc": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -202,6 +203,18 @@ def topk(H: int, G: int, n: int, k: int, scores=None, cand=None, out=None, works
     _check(lib().fathom_topk(_p(scores), _p(cand), H, G, n, int(k), _p(idx), _p(uni), _p(cnt), _p(workspace),
                              ws_bytes, _stream(stream)), "fathom_topk")
     return idx, uni, cnt
+
+
+def dequant_rows(planes, scales, n: int, rows, row_count=None, bits: int = 4, out=None, stream=None):
+    """Key rows rebuilt from the index: fp32 [H][M][D] for rows int32 [H][M]
+    (e.g. the union of ``topk``), at ``bits`` planes."""
+    H, D = planes.shape[0], planes.shape[1]
+    M = rows.shape[1]
+    if out is None:
+        out = torch.empty((H, M, D), dtype=torch.float32, device=rows.device)
+    _check(lib().fathom_dequant_rows(_p(planes), _p(scales), H, D, n, planes.shape[-1], _p(rows), M,
+                                     _p(row_count), int(bits), _p(out), _stream(stream)), "fathom_dequant_rows")
+    return out
 
 
 def scan_topk_noalloc(planes, scales, n: int, active, n_active, q, k: int, out=None, stream=None):

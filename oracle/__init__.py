@@ -48,6 +48,8 @@ def _lib():
         lib.orc_scan.argtypes = [P, P, I64, I, I64, I64, P, P, I, P, P]
         lib.orc_topk.restype = I
         lib.orc_topk.argtypes = [P, I64, I, I64, I, P, P, P]
+        lib.orc_dequant_rows.restype = I
+        lib.orc_dequant_rows.argtypes = [P, P, I64, I, I64, I64, P, I64, P, I, P]
         _LIB = lib
     return _LIB
 
@@ -168,3 +170,17 @@ def topk(scores: np.ndarray, k: int):
     cnt = np.zeros(H, dtype=np.int32)
     _check(_lib().orc_topk(_ptr(scores), H, G, n, int(k), _ptr(idx), _ptr(uni), _ptr(cnt)), "topk")
     return idx, uni, cnt
+
+
+def dequant_rows(planes: np.ndarray, scales: np.ndarray, n: int, rows: np.ndarray, row_count=None, bits: int = 4):
+    """fp64 key rows [H][M][D] rebuilt from the planes at ``bits`` planes."""
+    planes = np.ascontiguousarray(planes, dtype=np.uint64)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    H, D = planes.shape[0], planes.shape[1]
+    M = rows.shape[1]
+    rc = None if row_count is None else np.ascontiguousarray(row_count, dtype=np.int32)
+    out = np.zeros((H, M, D), dtype=np.float64)
+    _check(_lib().orc_dequant_rows(_ptr(planes), _ptr(scales), H, D, n, planes.shape[-1], _ptr(rows), M,
+                                   None if rc is None else _ptr(rc), int(bits), _ptr(out)), "dequant_rows")
+    return out

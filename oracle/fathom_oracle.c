@@ -26,6 +26,8 @@
  *                      paragraph: one plan shared by the G heads)
  *   orc_topk           full sort per query head + union per KV head
  *                      (byte-accounting section, top-k bullet)
+ *   orc_dequant_rows   whole key rows rebuilt from the planes (limits
+ *                      section, storage-overhead paragraph)
  */
 #include <math.h>
 #include <stdint.h>
@@ -374,5 +376,38 @@ int orc_topk(const double* scores, int64_t H, int G, int64_t n, int k,
     }
     free(c);
     free(u);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Key rows rebuilt from the stored planes: for list entry r of group h */
+/* (token i = rows[h*M + r]) and channel j, the `bits`-plane prefix     */
+/* value of the stored code.  Entries outside [0, n), and entries past  */
+/* row_count[h] (a negative count reads as 0), give 0.                  */
+/* ------------------------------------------------------------------ */
+int orc_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n,
+                     int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count,
+                     int bits, double* out)
+{
+    if (!planes || !scales || !rows || !out || H < 0 || D <= 0 || M < 0 || bits < 1 || bits > 4)
+        return ORC_EINVAL;
+    for (int64_t h = 0; h < H; ++h) {
+        int64_t count = M;
+        if (row_count) count = row_count[h] < 0 ? 0 : (row_count[h] > M ? M : row_count[h]);
+        for (int64_t r = 0; r < M; ++r) {
+            int64_t i = rows[h * M + r];
+            for (int j = 0; j < D; ++j) {
+                double v = 0.0;
+                if (r < count && i >= 0 && i < n) {
+                    int64_t b = i / 64;
+                    int c4 = 0;
+                    for (int p = 0; p < 4; ++p)
+                        if ((planes[(((h * D) + j) * 4 + p) * nb_stride + b] >> (i % 64)) & 1) c4 |= 1 << (3 - p);
+                    v = orc_dequant(c4, bits, orc_fp16_value(scales[(h * D + j) * nb_stride + b]));
+                }
+                out[(h * M + r) * D + j] = v;
+            }
+        }
+    }
     return ORC_OK;
 }

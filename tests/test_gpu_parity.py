@@ -230,3 +230,40 @@ def test_rotated_basis_full_path(fathom_gpu, orc):
     ref, l1 = orc.scan(p_ref, s_ref, d_ref, qr.cpu().numpy(), w.n)
     assert_scores_close(sc.cpu().numpy(), ref, l1)
     assert_topk_sets_match(idx.cpu().numpy(), orc.topk(ref, w.k)[0], ref, l1, w.k)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_dequant_rows_bit_exact(fathom_gpu, orc, bits):
+    w = dataclasses.replace(inputs.LAYER_32K, H=3, n=9000, seed=71)
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    rng = np.random.default_rng(bits)
+    M = 300
+    rows = np.sort(rng.integers(-5, w.n + 5, (w.H, M)), axis=1).astype(np.int32)
+    count = np.array([M, 123, -6], np.int32)          # full, partial, flagged group
+    out = fathom_gpu.dequant_rows(planes, scales, w.n, torch.tensor(rows, device=DEV),
+                                  torch.tensor(count, device=DEV), bits=bits)
+    torch.cuda.synchronize()
+    p_ref, s_ref = oracle_pack(orc, k, planes.shape[-1])
+    ref = orc.dequant_rows(p_ref, s_ref, w.n, rows, count, bits)
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), ref)
+
+
+def test_dequant_rows_of_the_union(fathom_gpu, orc):
+    """The winners' keys, rebuilt from the planes for the union a step returns."""
+    w = inputs.LAYER_32K
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    idx, uni, cnt = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, budget=48).run(q)
+    out = fathom_gpu.dequant_rows(planes, scales, w.n, uni, cnt)
+    torch.cuda.synchronize()
+    p_ref, s_ref = oracle_pack(orc, k, planes.shape[-1])
+    ref = orc.dequant_rows(p_ref, s_ref, w.n, uni.cpu().numpy(), cnt.cpu().numpy(), 4)
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), ref)
+    # the 4-plane rows are the keys' 4-bit values: within half a cell of the key
+    kk = k.float().cpu().numpy()
+    for h in range(w.H):
+        u = uni[h, :cnt[h]].cpu().numpy()
+        err = np.abs(out[h, :len(u)].cpu().numpy() - kk[h, u])
+        s = np.array([[orc.fp16_value(int(x)) for x in row] for row in s_ref[h][:, u // 64].T])
+        assert np.all(err <= s / 16 + 1e-7)

@@ -452,3 +452,27 @@ def test_byte_accounting_matches_printed_figures():
     check("a100_int_ops_per_hbm_byte", 108 * 64 * 1.41e9 / 2.0e12)
     # the scan-byte helper agrees with the per-token figure
     assert acc.scan_bytes(2 ** 20, 48, 32, query_bytes=False) * 8 / 2 ** 20 == acc.read_bits_per_token(48, 32)
+
+
+# --------------------------------------------------------------------------
+# Key rows rebuilt from the planes (section 边界, storage-overhead paragraph)
+# --------------------------------------------------------------------------
+def test_dequant_rows_is_the_midrise_value_of_each_key(orc):
+    rng = np.random.default_rng(16)
+    H, n, D = 2, 300, 16
+    keys = (rng.standard_normal((H, n, D)) * 3).astype(np.float32)
+    planes, scales = orc.pack(keys)
+    M = 40
+    rows = rng.integers(-3, n + 3, (H, M)).astype(np.int32)   # includes out-of-range entries
+    count = np.array([M, 25], np.int32)
+    for bits in range(1, 5):
+        out = orc.dequant_rows(planes, scales, n, rows, count, bits)
+        for h in range(H):
+            for r in range(M):
+                i = rows[h, r]
+                for j in range(D):
+                    if r >= count[h] or not 0 <= i < n:
+                        assert out[h, r, j] == 0.0
+                        continue
+                    s = Fraction(orc.fp16_value(int(scales[h, j, i // 64])))
+                    assert Fraction(out[h, r, j]) == midrise(Fraction(float(keys[h, i, j])), bits, s)
