@@ -103,6 +103,13 @@ int64_t fathom_nb_stride(int64_t n);
  *   scales      DEVICE out, fp16 bit patterns [H][D][nb_stride].
  *   nb_stride   words per plane row, >= ceil(n/64) and even.
  * Words/scales at block indices >= ceil(n/64) are not written.
+ *
+ * Appending during decode: new tokens land in the tail block, whose scale
+ * (its maximum) can change, so the tail block is quantised again from its
+ * raw keys.  Call fathom_pack on the keys from token 64*b0 onwards with
+ * planes + b0 and scales + b0 (same nb_stride as the whole index): blocks
+ * b0.. are rewritten, earlier blocks are untouched, and the result equals
+ * packing all tokens at once.
  */
 int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
                 int64_t key_stride_h, int64_t key_stride_tok,

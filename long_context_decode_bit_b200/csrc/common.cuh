@@ -69,7 +69,11 @@ struct CandLayout {
     size_t off_hdr, off_sample, off_counts, off_entries, total;
 };
 
-constexpr int kScanTileBlocks = 16;                       // 1024 tokens per scan tile
+#ifndef FATHOM_SCAN_TILE_BLOCKS
+#define FATHOM_SCAN_TILE_BLOCKS 32
+#endif
+constexpr int kScanTileBlocks = FATHOM_SCAN_TILE_BLOCKS;   // 64-token blocks per scan tile (16 or 32)
+static_assert(kScanTileBlocks == 16 || kScanTileBlocks == 32, "scan tiles hold 16 or 32 blocks");
 constexpr int kScanTileTokens = kScanTileBlocks * kBlockTokens;
 
 CandLayout cand_layout(int64_t H, int G, int64_t n, int k);

@@ -42,13 +42,13 @@ namespace fathom {
 
 namespace {
 
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = kScanTileBlocks / 4;            // each consumer warp owns 4 blocks
 constexpr int kScanThreads = 32 * (kConsumerWarps + 1);         // + one producer warp
 constexpr int kBlocksPerWarp = kScanTileBlocks / kConsumerWarps;  // 4
 constexpr int kStages = 3;   // the stage_sync/stage_arrive helpers spell out 3 stages
 constexpr int kChunkCh = 40;        // channels per chunk
 constexpr int kChunkRows = 64;      // plane rows per chunk
-constexpr int kRowBytes = kScanTileBlocks * 8;   // one plane row of a tile: 128 B
+constexpr int kRowBytes = kScanTileBlocks * 8;   // one plane row of a tile: 128 or 256 B
 
 // Named barriers (0 is __syncthreads).
 constexpr int kBarReady = 1;                 // + stage: producer -> consumers
@@ -246,7 +246,7 @@ __device__ __forceinline__ float acc_at(const float2 (&acc)[8][head_pairs<G>()],
 }
 
 #ifndef FATHOM_SCAN_MIN_CTAS
-#define FATHOM_SCAN_MIN_CTAS 3
+#define FATHOM_SCAN_MIN_CTAS (kScanTileBlocks == 16 ? 3 : 2)
 #endif
 #ifndef FATHOM_SCAN_TILES_CAP
 #define FATHOM_SCAN_TILES_CAP 32
@@ -364,9 +364,10 @@ scan_kernel(const ScanArgs a)
             const int64_t valid_blocks = a.nb - b0;   // >= 1
             const int r0 = S.chunk_row0[ck], rows = S.chunk_row0[ck + 1] - r0;
             const int c0 = S.chunk_begin[ck], nc = S.chunk_begin[ck + 1] - c0;
-            // Plane rows: 8 pieces of 16 B (2 blocks each) per row.
-            for (int idx = lane; idx < rows * 8; idx += 32) {
-                const int r = idx >> 3, part = idx & 7;
+            // Plane rows: pieces of 16 B (2 blocks each), kScanTileBlocks / 2 per row.
+            constexpr int kRowPieces = kScanTileBlocks / 2;
+            for (int idx = lane; idx < rows * kRowPieces; idx += 32) {
+                const int r = idx / kRowPieces, part = idx % kRowPieces;
                 const int src_rc = S.rowsrc[r0 + r];
                 const int64_t row = (h * D + (src_rc >> 2)) * kPlanes + (src_rc & 3);
                 const int64_t vb = valid_blocks - 2 * part;
@@ -374,9 +375,10 @@ scan_kernel(const ScanArgs a)
                 const uint64_t* src = a.planes + row * a.nb_stride + (bytes ? b0 + 2 * part : 0);
                 cp_async16(&S.words[st][r * kScanTileBlocks + 2 * part], src, bytes);
             }
-            // Scale rows: 2 pieces of 16 B (8 blocks each) per channel.
-            for (int idx = lane; idx < nc * 2; idx += 32) {
-                const int c = idx >> 1, part = idx & 1;
+            // Scale rows: pieces of 16 B (8 blocks each), kScanTileBlocks / 8 per channel.
+            constexpr int kScalePieces = kScanTileBlocks / 8;
+            for (int idx = lane; idx < nc * kScalePieces; idx += 32) {
+                const int c = idx / kScalePieces, part = idx % kScalePieces;
                 const int j = S.chan[c0 + c] & 0xFF;
                 const int64_t vb = valid_blocks - 8 * part;
                 const int bytes = vb >= 8 ? 16 : (vb > 0 ? static_cast<int>(vb) * 2 : 0);

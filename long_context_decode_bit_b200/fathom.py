@@ -52,11 +52,13 @@ class FathomError(RuntimeError):
         super().__init__(msg)
 
 
-def load(path: str = LIB_PATH):
-    """Load the shared library (raises if it is missing)."""
+def load(path: str | None = None):
+    """Load the shared library (raises if it is missing).  ``FATHOM_LIB``
+    may name another build of it."""
     global _lib
     if _lib is not None:
         return _lib
+    path = path or os.environ.get("FATHOM_LIB") or LIB_PATH
     if not os.path.exists(path):
         raise FileNotFoundError(
             f"{path} is missing: build it with `python -m long_context_decode_bit_b200.build`")
@@ -130,6 +132,24 @@ def pack(keys: torch.Tensor, nb_stride_words: int | None = None, planes=None, sc
         scales = torch.zeros((H, D, nbs), dtype=torch.int16, device=dev)
     _check(lib().fathom_pack(_p(keys), dt, H, n, D, keys.stride(0), keys.stride(1), _p(planes), _p(scales),
                              nbs, _stream(stream)), "fathom_pack")
+    return planes, scales
+
+
+def pack_range(keys: torch.Tensor, planes: torch.Tensor, scales: torch.Tensor, block0: int, stream=None):
+    """(Re)pack blocks block0.. of an existing index from ``keys`` [H][m][D],
+    the keys of tokens 64*block0 .. 64*block0 + m - 1 (appending to the tail
+    block during decode).  ``planes``/``scales`` are the whole index."""
+    H, m, D = keys.shape
+    if keys.stride(2) != 1:
+        raise ValueError("keys must be contiguous along channels")
+    dt = {torch.float32: KEYS_F32, torch.bfloat16: KEYS_BF16}[keys.dtype]
+    nbs = planes.shape[-1]
+    if block0 < 0 or block0 + (m + 63) // 64 > nbs:
+        raise ValueError("block range outside the index")
+    pp = ctypes.c_void_p(planes.data_ptr() + 8 * block0)
+    sp = ctypes.c_void_p(scales.data_ptr() + 2 * block0)
+    _check(lib().fathom_pack(_p(keys), dt, H, m, D, keys.stride(0), keys.stride(1), pp, sp, nbs, _stream(stream)),
+           "fathom_pack")
     return planes, scales
 
 

@@ -50,10 +50,10 @@ def test_host_only_entry_points(lib):
     small = lib.fathom_scan_cand_bytes(2, 4, 1000, 64)        # no sample: cap = n
     assert small >= 2 * 4 * (16 + 1000 * 8)
     big = lib.fathom_scan_cand_bytes(288, 4, 2 ** 20, 512)
-    # 1152 heads x (1024 tiles x 16 survivor slots of 8 B + 1024 tile counts
-    # + 32768 sample scores of 4 B) + headers
-    per_head = 1024 * 16 * 8 + 1024 * 4 + 32768 * 4
-    assert 1152 * per_head <= big < 1152 * (per_head + 16) + 4 * 256
+    # 1152 heads x (16384 survivor slots of 8 B, i.e. 8x the ~2048 expected,
+    # spread over the tiles + one count per tile + 32768 sample scores of 4 B)
+    per_head = 16384 * 8 + 32768 * 4
+    assert 1152 * per_head <= big < 1152 * (per_head + 4096 + 16) + 4 * 256
 
 
 def test_rejections_before_any_cuda_call(lib):

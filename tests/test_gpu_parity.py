@@ -267,3 +267,28 @@ def test_dequant_rows_of_the_union(fathom_gpu, orc):
         err = np.abs(out[h, :len(u)].cpu().numpy() - kk[h, u])
         s = np.array([[orc.fp16_value(int(x)) for x in row] for row in s_ref[h][:, u // 64].T])
         assert np.all(err <= s / 16 + 1e-7)
+
+
+def test_append_repacks_the_tail_block(fathom_gpu, orc):
+    """Decode-time append: tokens arrive one small batch at a time; each time
+    the tail block is packed again from its raw keys.  The index must equal
+    packing every token at once (and so the oracle's)."""
+    w = dataclasses.replace(inputs.LAYER_32K, H=3, n=5200, seed=81)
+    k, _, _ = make(w)
+    n_max = w.n
+    nbs = fathom_gpu.nb_stride(n_max)
+    planes = torch.zeros((w.H, w.D, 4, nbs), dtype=torch.int64, device=DEV)
+    scales = torch.zeros((w.H, w.D, nbs), dtype=torch.int16, device=DEV)
+    n = 4990
+    fathom_gpu.pack_range(k[:, :n].contiguous(), planes, scales, 0)
+    for step in (1, 5, 64, 70, 3, 67):            # crosses several block boundaries
+        n_new = min(n_max, n + step)
+        b0 = n // 64                              # the block holding token n (the old tail)
+        fathom_gpu.pack_range(k[:, b0 * 64:n_new].contiguous(), planes, scales, b0)
+        n = n_new
+    torch.cuda.synchronize()
+    full_p, full_s = fathom_gpu.pack(k[:, :n].contiguous(), nb_stride_words=nbs)
+    torch.cuda.synchronize()
+    assert torch.equal(planes, full_p) and torch.equal(scales, full_s)
+    p_ref, s_ref = orc.pack(keys_for_oracle(k[:, :n]), nb_stride=nbs)
+    assert np.array_equal(np_u64(planes), p_ref) and np.array_equal(np_u16(scales), s_ref)
