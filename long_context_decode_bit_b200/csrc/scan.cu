@@ -50,6 +50,11 @@ constexpr int kChunkCh = 40;        // channels per chunk
 constexpr int kChunkRows = 64;      // plane rows per chunk
 constexpr int kRowBytes = kScanTileBlocks * 8;   // one plane row of a tile: 128 or 256 B
 
+#ifndef FATHOM_SCAN_TILES_CAP
+#define FATHOM_SCAN_TILES_CAP 32
+#endif
+constexpr int kMaxTilesPerCta = FATHOM_SCAN_TILES_CAP;
+
 // Named barriers (0 is __syncthreads).
 constexpr int kBarReady = 1;                 // + stage: producer -> consumers
 constexpr int kBarEmpty = 1 + kStages;       // + stage: consumers -> producer
@@ -98,7 +103,7 @@ struct SharedScan {
     int n_chunks;
     float tau[G];
     int direct[G];                   // no threshold sample: every key is kept, at its own index
-    int tile_cnt[G];                 // survivors of the current tile per head
+    int tile_cnt[kMaxTilesPerCta][G];// survivors per (tile of this CTA, head), written out at the end
 };
 
 // Named barriers with compile-time ids (a run-time id reserves all 16).
@@ -248,9 +253,6 @@ __device__ __forceinline__ float acc_at(const float2 (&acc)[8][head_pairs<G>()],
 #ifndef FATHOM_SCAN_MIN_CTAS
 #define FATHOM_SCAN_MIN_CTAS (kScanTileBlocks == 16 ? 3 : 2)
 #endif
-#ifndef FATHOM_SCAN_TILES_CAP
-#define FATHOM_SCAN_TILES_CAP 32
-#endif
 
 template <int G>
 __global__ void __launch_bounds__(kScanThreads, FATHOM_SCAN_MIN_CTAS)
@@ -340,8 +342,8 @@ scan_kernel(const ScanArgs a)
     if (a.mode == kCandidate && tid < G) {
         S.tau[tid] = a.hdr[h * G + tid].tau;
         S.direct[tid] = a.hdr[h * G + tid].n_sample == 0;
-        S.tile_cnt[tid] = 0;
     }
+    for (int i = tid; i < kMaxTilesPerCta * G; i += kScanThreads) (&S.tile_cnt[0][0])[i] = 0;
     __syncthreads();   // plan, coefficients' q part and thresholds visible to every warp
 
     // Tiles of this CTA that exist.
@@ -486,22 +488,24 @@ scan_kernel(const ScanArgs a)
                             if (S.direct[g]) {
                                 a.entries[(h * G + g) * a.cap + i] = ent;
                             } else {
-                                const int p = atomicAdd(&S.tile_cnt[g], 1);
+                                const int p = atomicAdd(&S.tile_cnt[ti][g], 1);
                                 if (p < a.tslot) a.entries[(h * G + g) * a.cap + ptile * a.tslot + p] = ent;
                             }
                         }
                     }
                 }
-                if (a.tslot > 0) {
-                    bar_sync<kBarConsumers, 32 * kConsumerWarps>();   // every consumer warp has appended
-                    if (tid < G) {
-                        a.tile_counts[(h * G + tid) * a.tiles + ptile] = S.tile_cnt[tid];
-                        S.tile_cnt[tid] = 0;
-                    }
-                }
             }
         }
         if (u + kStages < units) stage_arrive<kBarEmpty>(st);   // stage st may be refilled
+    }
+    // Survivor counts of every tile of this CTA, once all consumer warps are done.
+    if (a.mode == kCandidate && a.tslot > 0) {
+        bar_sync<kBarConsumers, 32 * kConsumerWarps>();
+        for (int i = tid; i < tiles_here * G; i += 32 * kConsumerWarps) {
+            const int ti = i / G, g = i % G;
+            const int64_t ptile = (static_cast<int64_t>(blockIdx.x) * a.tiles_per_cta + ti) * a.tile_stride;
+            a.tile_counts[(h * G + g) * a.tiles + ptile] = S.tile_cnt[ti][g];
+        }
     }
 }
 
