@@ -48,7 +48,7 @@ typedef struct CUstream_st* fathom_stream_t; /* same type as cudaStream_t */
 #define FATHOM_ERR_UNSUPPORTED (-2) /* D, G, k or alignment outside the limits above */
 #define FATHOM_ERR_CUDA (-3)        /* a CUDA call failed; see fathom_last_cuda_error() */
 #define FATHOM_ERR_WORKSPACE (-4)   /* caller buffer smaller than the *_bytes() query */
-#define FATHOM_ERR_TIMEOUT (-5)     /* reserved: a bounded device wait gave up */
+#define FATHOM_ERR_TIMEOUT (-5)     /* a bounded device wait gave up; see fathom_device_status() */
 #define FATHOM_ERR_OVERFLOW (-6)    /* candidate pass could not prove its top-k exact */
 
 /* Key element types for fathom_pack. */
@@ -214,6 +214,12 @@ size_t fathom_scan_cand_bytes(int64_t H, int G, int64_t n, int k);
  *                   DENSE, which ignores it), 16-byte aligned.
  *   k               winners per query head that will be asked of
  *                   fathom_topk (sizes the candidate pass).
+ *
+ * The kernel hands plane rows from a loader warp to the compute warps
+ * through a shared-memory ring whose waits are bounded.  A wait that gives
+ * up (which a correct launch never does) sets the device fault word and
+ * the launch's outputs are void: fathom_topk then reports
+ * FATHOM_ERR_TIMEOUT, and fathom_device_status() returns it.
  */
 int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D,
                 int64_t n, int64_t nb_stride, const uint16_t* active,
@@ -243,7 +249,9 @@ size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k);
  *              FATHOM_ERR_OVERFLOW for a group whose candidate pass kept
  *              fewer than k or more than its capacity of keys; such a
  *              group's idx and union_idx are unspecified and the caller
- *              reruns it with a DENSE scan.
+ *              reruns it with a DENSE scan; FATHOM_ERR_TIMEOUT for every
+ *              group while the device fault word is set (a scan's bounded
+ *              wait gave up: nothing of that step is valid).
  *   workspace, ws_bytes  DEVICE scratch of fathom_topk_workspace_bytes()
  *              bytes (may be NULL when that is 0).
  */
@@ -311,6 +319,20 @@ int fathom_scan_topk_noalloc(const uint64_t* planes, const uint16_t* scales, int
                              const int32_t* n_active, const float* q, int G, int k,
                              int32_t* idx, int32_t* union_idx, int32_t* union_count,
                              fathom_stream_t stream);
+
+/*
+ * fathom_device_status -- FATHOM_ERR_TIMEOUT if a kernel of this library on
+ * the current device has given up a bounded wait since the word was last
+ * cleared, else FATHOM_OK (or FATHOM_ERR_CUDA).  (The paper has no
+ * counterpart: this is the library's own failure report.)
+ *
+ * Reads the device's fault word in stream order and synchronises `stream`;
+ * with clear != 0 a set word is reset to 0 afterwards.  The word is one per
+ * device and process, so a fault seen here may come from work on another
+ * stream.  The first call on a device looks the word's address up (a
+ * one-time cudaGetSymbolAddress), as the first scan on that device does.
+ */
+int fathom_device_status(int clear, fathom_stream_t stream);
 
 #ifdef __cplusplus
 }

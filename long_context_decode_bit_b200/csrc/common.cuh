@@ -25,6 +25,10 @@ int cuda_status(cudaError_t e);
 // Launch-error check after a <<<>>> launch.
 inline int launch_status() { return cuda_status(cudaGetLastError()); }
 
+// Device address of this device's fault word (set when a bounded device
+// wait gave up; see fault.cu).
+int device_fault_word(int32_t** out);
+
 // ---------------------------------------------------------------------
 // Order-preserving map from fp32 to uint32: larger float -> larger key.
 // -0 is folded onto +0 so that the two compare equal, as fp32 values do.

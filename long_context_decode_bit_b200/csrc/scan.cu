@@ -6,13 +6,17 @@
 // where c_t is the key's t-bit prefix code read from the first t plane rows
 // of channel j.  The K bytes are read once for all G heads.
 //
-// Work layout.  A CTA is one producer warp and four consumer warps working
-// on one group.  The CTA walks `tiles_per_cta` tiles of 16 64-token blocks;
-// the group's active channels (sorted by depth once per CTA) are split into
-// chunks, and one (tile, chunk) pair is a pipeline unit.
-//   - The producer streams each unit's plane rows (16 words, 128 B per row)
-//     and fp16 scale rows into a 3-stage shared-memory ring with 16-byte
-//     cp.async copies, and hands stages over through named barriers.
+// Work layout.  A CTA is one producer warp and kScanTileBlocks / 4 consumer
+// warps working on one group.  The CTA walks `tiles_per_cta` tiles of
+// kScanTileBlocks 64-token blocks; the group's active channels (sorted by
+// depth once per CTA) are split into chunks, and one (tile, chunk) pair is a
+// pipeline unit.
+//   - The producer streams each unit's plane rows (one 64-bit word per
+//     block, 8 * kScanTileBlocks bytes per row) and fp16 scale rows into a
+//     3-stage shared-memory ring with 16-byte cp.async copies.  The copies'
+//     completion arrives on the stage's "full" mbarrier; each consumer warp
+//     arrives on its "empty" mbarrier when done, so a warp waits only for
+//     the data it needs, never for the other consumer warps.
 //   - Consumer warp w owns blocks 4w..4w+3 of a tile; a lane owns 8 tokens
 //     of one block: bit positions l, l+8, l+16, l+24 (l = lane & 7) of the
 //     block's low and of its high 32-bit plane half.  Each warp first forms
@@ -45,7 +49,7 @@ namespace {
 constexpr int kConsumerWarps = kScanTileBlocks / 4;            // each consumer warp owns 4 blocks
 constexpr int kScanThreads = 32 * (kConsumerWarps + 1);         // + one producer warp
 constexpr int kBlocksPerWarp = kScanTileBlocks / kConsumerWarps;  // 4
-constexpr int kStages = 3;   // the stage_sync/stage_arrive helpers spell out 3 stages
+constexpr int kStages = 3;
 constexpr int kChunkCh = 40;        // channels per chunk
 constexpr int kChunkRows = 64;      // plane rows per chunk
 constexpr int kRowBytes = kScanTileBlocks * 8;   // one plane row of a tile: 128 or 256 B
@@ -55,10 +59,11 @@ constexpr int kRowBytes = kScanTileBlocks * 8;   // one plane row of a tile: 128
 #endif
 constexpr int kMaxTilesPerCta = FATHOM_SCAN_TILES_CAP;
 
-// Named barriers (0 is __syncthreads).
-constexpr int kBarReady = 1;                 // + stage: producer -> consumers
-constexpr int kBarEmpty = 1 + kStages;       // + stage: consumers -> producer
-constexpr int kBarConsumers = 1 + 2 * kStages;
+// Named barrier among the consumer warps (0 is __syncthreads).
+constexpr int kBarConsumers = 1;
+// Upper bound on the polls of one ring wait; a wait that runs out marks the
+// launch faulty and the warp leaves its loop instead of spinning for ever.
+constexpr int kSpinLimit = 1 << 22;
 
 enum ScanMode { kDense = 0, kSample = 1, kCandidate = 2 };
 
@@ -78,6 +83,7 @@ struct ScanArgs {
     int64_t cap, tslot, n_sample, tile_stride, tiles;
     int tiles_per_cta;
     int mode;
+    int32_t* fault;            // device fault word: set when a ring wait ran out
 };
 
 // Heads are handled in pairs for the packed FMA; odd G gets a zero pad.
@@ -104,6 +110,8 @@ struct SharedScan {
     float tau[G];
     int direct[G];                   // no threshold sample: every key is kept, at its own index
     int tile_cnt[kMaxTilesPerCta][G];// survivors per (tile of this CTA, head), written out at the end
+    __align__(8) uint64_t full[kStages];   // ring: data of the stage has landed (32 producer lanes)
+    __align__(8) uint64_t empty[kStages];  // ring: every consumer warp is done with the stage
 };
 
 // Named barriers with compile-time ids (a run-time id reserves all 16).
@@ -119,20 +127,34 @@ __device__ __forceinline__ void bar_arrive()
     asm volatile("bar.arrive %0, %1;\n" ::"n"(ID), "n"(COUNT) : "memory");
 }
 
-template <int BASE>
-__device__ __forceinline__ void stage_sync(int st)
+__device__ __forceinline__ void mbar_init(uint32_t bar, int count)
 {
-    if (st == 0) bar_sync<BASE + 0, kScanThreads>();
-    else if (st == 1) bar_sync<BASE + 1, kScanThreads>();
-    else bar_sync<BASE + 2, kScanThreads>();
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
 }
 
-template <int BASE>
-__device__ __forceinline__ void stage_arrive(int st)
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
 {
-    if (st == 0) bar_arrive<BASE + 0, kScanThreads>();
-    else if (st == 1) bar_arrive<BASE + 1, kScanThreads>();
-    else bar_arrive<BASE + 2, kScanThreads>();
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar) : "memory");
+}
+
+// One arrival on `bar` once every cp.async this thread has issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+
+// Wait for the phase of `bar` with the given parity to complete; false if
+// the poll limit ran out first.  Each poll suspends the thread for at most
+// about a microsecond, so a wait gives up after a few seconds at most.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    for (int it = 0; it < kSpinLimit; ++it) {
+        uint32_t ok;
+        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+                     : "=r"(ok) : "r"(bar), "r"(parity), "n"(1000) : "memory");
+        if (ok) return true;
+    }
+    return false;
 }
 
 // 16-byte copy of which only the first `bytes` (0..16) are read; the rest is zero-filled.
@@ -142,10 +164,7 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int byt
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 // Depth-1 values of the four tokens of one 32-bit half: +-1.0f.
 __device__ __forceinline__ void values_depth1(uint32_t w, int l, float (&v)[4])
@@ -172,6 +191,14 @@ __device__ __forceinline__ void values_depth(const uint32_t (&w)[4], int l, floa
 #pragma unroll
     for (int m = 0; m < 4; ++m)   // exact odd integers
         v[m] = __fmaf_rn(__uint_as_float(__byte_perm(code, 0x4B400000u, 0x7650u + m)), mul, -sub);
+}
+
+// max(a, b, c) in one instruction (NaN operands are dropped, as fmaxf drops them).
+__device__ __forceinline__ float max3f(float x, float y, float z)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(x), "f"(y), "f"(z));
+    return r;
 }
 
 __device__ __forceinline__ uint2 lds_u2(uint32_t addr)
@@ -344,7 +371,13 @@ scan_kernel(const ScanArgs a)
         S.direct[tid] = a.hdr[h * G + tid].n_sample == 0;
     }
     for (int i = tid; i < kMaxTilesPerCta * G; i += kScanThreads) (&S.tile_cnt[0][0])[i] = 0;
-    __syncthreads();   // plan, coefficients' q part and thresholds visible to every warp
+    if (tid < kStages) {
+        mbar_init(static_cast<uint32_t>(__cvta_generic_to_shared(&S.full[tid])), 32);
+        mbar_init(static_cast<uint32_t>(__cvta_generic_to_shared(&S.empty[tid])), kConsumerWarps);
+    }
+    __syncthreads();   // plan, coefficients' q part, thresholds and ring barriers visible to every warp
+    const uint32_t full0 = static_cast<uint32_t>(__cvta_generic_to_shared(&S.full[0]));
+    const uint32_t empty0 = static_cast<uint32_t>(__cvta_generic_to_shared(&S.empty[0]));
 
     // Tiles of this CTA that exist.
     int64_t tiles_here = a.tiles_per_cta;
@@ -359,7 +392,10 @@ scan_kernel(const ScanArgs a)
         // ================= producer warp =================
         for (int u = 0; u < units; ++u) {
             const int st = u % kStages;
-            if (u >= kStages) stage_sync<kBarEmpty>(st);   // consumers freed this stage
+            if (u >= kStages && !__all_sync(0xffffffffu, mbar_wait(empty0 + 8 * st, ((u / kStages) - 1) & 1))) {
+                if (lane == 0) atomicOr(a.fault, 1);   // consumers never freed this stage
+                break;
+            }
             const int ti = u / n_chunks, ck = u % n_chunks;
             const int64_t ltile = static_cast<int64_t>(blockIdx.x) * a.tiles_per_cta + ti;
             const int64_t b0 = ltile * a.tile_stride * kScanTileBlocks;
@@ -387,16 +423,9 @@ scan_kernel(const ScanArgs a)
                 const uint16_t* src = a.scales + (h * D + j) * a.nb_stride + (bytes ? b0 + 8 * part : 0);
                 cp_async16(&S.rawscale[st][c * kScanTileBlocks + 8 * part], src, bytes);
             }
-            cp_async_commit();
-            if (u >= 1) {
-                cp_async_wait<1>();   // unit u-1 has landed
-                stage_arrive<kBarReady>((u - 1) % kStages);
-            }
+            cp_async_arrive(full0 + 8 * st);   // this lane's share of unit u
         }
-        if (units >= 1) {
-            cp_async_wait<0>();
-            stage_arrive<kBarReady>((units - 1) % kStages);
-        }
+        cp_async_wait_all();
         return;
     }
 
@@ -410,7 +439,10 @@ scan_kernel(const ScanArgs a)
     for (int u = 0; u < units; ++u) {
         const int st = u % kStages;
         const int ti = u / n_chunks, ck = u % n_chunks;
-        stage_sync<kBarReady>(st);   // unit u is in stage st
+        if (!__all_sync(0xffffffffu, mbar_wait(full0 + 8 * st, (u / kStages) & 1))) {   // unit u is in stage st
+            if (lane == 0) atomicOr(a.fault, 1);
+            break;
+        }
 
         const int c0 = S.chunk_begin[ck], nc = S.chunk_begin[ck + 1] - c0;
         // Coefficients of the warp's 4 blocks: (channel, block) -> G/2 head pairs.
@@ -467,36 +499,35 @@ scan_kernel(const ScanArgs a)
                 }
             } else {
                 const int64_t ptile = ltile * a.tile_stride;
-                // Most lanes hold no survivor: test each head's maximum first.
-                bool any = false;
+                // Most lanes hold no survivor: a head's 8 scores are tested
+                // one by one only when their maximum reaches its threshold.
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    float mx = acc_at<G>(acc, 0, g);
+                    const float tau = S.tau[g];
+                    const float mx = max3f(max3f(acc_at<G>(acc, 0, g), acc_at<G>(acc, 1, g), acc_at<G>(acc, 2, g)),
+                                           max3f(acc_at<G>(acc, 3, g), acc_at<G>(acc, 4, g), acc_at<G>(acc, 5, g)),
+                                           fmaxf(acc_at<G>(acc, 6, g), acc_at<G>(acc, 7, g)));
+                    if (mx >= tau) {
 #pragma unroll
-                    for (int m = 1; m < 8; ++m) mx = fmaxf(mx, acc_at<G>(acc, m, g));
-                    any |= mx >= S.tau[g];
-                }
-                if (any)
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int64_t i = tok0 + (m >> 2) * 32 + 8 * (m & 3);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        const float sv = acc_at<G>(acc, m, g);
-                        if (i < a.n && sv >= S.tau[g]) {
-                            const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
-                            if (S.direct[g]) {
-                                a.entries[(h * G + g) * a.cap + i] = ent;
-                            } else {
-                                const int p = atomicAdd(&S.tile_cnt[ti][g], 1);
-                                if (p < a.tslot) a.entries[(h * G + g) * a.cap + ptile * a.tslot + p] = ent;
+                        for (int m = 0; m < 8; ++m) {
+                            const float sv = acc_at<G>(acc, m, g);
+                            const int64_t i = tok0 + (m >> 2) * 32 + 8 * (m & 3);
+                            if (sv >= tau && i < a.n) {
+                                const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
+                                if (S.direct[g]) {
+                                    a.entries[(h * G + g) * a.cap + i] = ent;
+                                } else {
+                                    const int p = atomicAdd(&S.tile_cnt[ti][g], 1);
+                                    if (p < a.tslot) a.entries[(h * G + g) * a.cap + ptile * a.tslot + p] = ent;
+                                }
                             }
                         }
                     }
                 }
             }
         }
-        if (u + kStages < units) stage_arrive<kBarEmpty>(st);   // stage st may be refilled
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * st);   // stage st may be refilled
     }
     // Survivor counts of every tile of this CTA, once all consumer warps are done.
     if (a.mode == kCandidate && a.tslot > 0) {
@@ -589,6 +620,10 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
                 int G, int mode, float* scores, void* cand, int k, cudaStream_t stream)
 {
     ScanArgs a{};
+    {
+        const int st = device_fault_word(&a.fault);
+        if (st) return st;
+    }
     a.planes = planes;
     a.scales = scales;
     a.nb_stride = nb_stride;

@@ -260,7 +260,7 @@ topk_kernel(const TopkArgs a)
 // Sorted, de-duplicated union of a group's G winner lists.
 __global__ void __launch_bounds__(kTopkThreads)
 union_kernel(const int32_t* __restrict__ idx, int G, int k, int upow2, int32_t* __restrict__ union_idx,
-             int32_t* __restrict__ union_count)
+             int32_t* __restrict__ union_count, const int32_t* __restrict__ fault)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     int32_t* v = reinterpret_cast<int32_t*>(smem);
@@ -278,9 +278,10 @@ union_kernel(const int32_t* __restrict__ idx, int G, int k, int upow2, int32_t* 
         v[i] = x;
     }
     __syncthreads();
-    if (failed) {
+    const int32_t faulted = *fault;   // a scan whose ring wait gave up left void scores
+    if (failed || faulted) {
         for (int i = tid; i < gk; i += blockDim.x) dst[i] = -1;
-        if (tid == 0) union_count[h] = FATHOM_ERR_OVERFLOW;
+        if (tid == 0) union_count[h] = faulted ? FATHOM_ERR_TIMEOUT : FATHOM_ERR_OVERFLOW;
         return;
     }
     bitonic_sort<int32_t, false>(v, upow2);
@@ -353,12 +354,15 @@ int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
     topk_kernel<<<dim3(G, static_cast<unsigned>(H)), kTopkThreads, smem, stream>>>(a);
     int st = launch_status();
     if (st) return st;
+    int32_t* fault = nullptr;
+    st = device_fault_word(&fault);
+    if (st) return st;
     const int upow2 = pow2_at_least(G * k);
     const size_t usmem = sizeof(int32_t) * upow2;
     e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(usmem));
     if (e != cudaSuccess) return cuda_status(e);
     union_kernel<<<static_cast<unsigned>(H), kTopkThreads, usmem, stream>>>(idx, G, k, upow2, union_idx,
-                                                                          union_count);
+                                                                          union_count, fault);
     return launch_status();
 }
 

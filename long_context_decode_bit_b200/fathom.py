@@ -36,6 +36,7 @@ EXPORTS = (
     "fathom_version", "fathom_status_string", "fathom_last_cuda_error", "fathom_nb_stride",
     "fathom_pack", "fathom_plan", "fathom_plan_fixed", "fathom_scan_cand_bytes", "fathom_scan",
     "fathom_topk_workspace_bytes", "fathom_topk", "fathom_dequant_rows", "fathom_scan_topk_noalloc",
+    "fathom_device_status",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -78,6 +79,7 @@ def load(path: str | None = None):
         "fathom_topk": (I, [P, P, I64, I, I64, I, P, P, P, P, SZ, P]),
         "fathom_dequant_rows": (I, [P, P, I64, I, I64, I64, P, I64, P, I, P, P]),
         "fathom_scan_topk_noalloc": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, P, P]),
+        "fathom_device_status": (I, [I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -255,6 +257,16 @@ def scan_topk_noalloc(planes, scales, n: int, active, n_active, q, k: int, out=N
     return idx, uni, cnt
 
 
+def device_status(clear: bool = False, stream=None) -> int:
+    """OK, or ERR_TIMEOUT if a library kernel on the current device gave up
+    a bounded wait since the fault word was last cleared (synchronises the
+    stream)."""
+    st = int(lib().fathom_device_status(1 if clear else 0, _stream(stream)))
+    if st not in (OK, ERR_TIMEOUT):
+        _check(st, "fathom_device_status")
+    return st
+
+
 class Step:
     """One decode step of the scan over a resident index: plan -> candidate
     scan -> top-k + union, with the dense rerun for any group whose
@@ -317,6 +329,8 @@ class Step:
         bad = torch.nonzero(cnt < 0).flatten().tolist()
         if not bad:
             return 0
+        if int(cnt[bad[0]]) == ERR_TIMEOUT:
+            raise FathomError(ERR_TIMEOUT, "candidate scan (device fault word set)")
         _, active, n_active, _ = self.plan_out
         for h in bad:
             sl = slice(h, h + 1)
