@@ -40,6 +40,8 @@
 // strided subset of tiles to the candidate buffer's sample area; CANDIDATE
 // keeps keys whose score reaches the head's threshold: at their own index
 // when there is no threshold sample, else in this tile's slot range.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace fathom {
@@ -193,14 +195,6 @@ __device__ __forceinline__ void values_depth(const uint32_t (&w)[4], int l, floa
         v[m] = __fmaf_rn(__uint_as_float(__byte_perm(code, 0x4B400000u, 0x7650u + m)), mul, -sub);
 }
 
-// max(a, b, c) in one instruction (NaN operands are dropped, as fmaxf drops them).
-__device__ __forceinline__ float max3f(float x, float y, float z)
-{
-    float r;
-    asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(x), "f"(y), "f"(z));
-    return r;
-}
-
 __device__ __forceinline__ uint2 lds_u2(uint32_t addr)
 {
     uint2 v;
@@ -225,8 +219,9 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr)
 // One channel of depth T for the lane's block: 8 tokens x G heads.
 // wrow: shared address of the channel's first plane row at the lane's block
 // column; cf: shared address of its head-pair coefficients for that block.
-template <int G, int T>
-__device__ __forceinline__ void channel_step(uint32_t wrow, uint32_t cf, int l, float2 (&acc)[8][head_pairs<G>()])
+// The 8 token values of one channel of depth T for the lane's block.
+template <int T>
+__device__ __forceinline__ void channel_values(uint32_t wrow, int l, float (&v)[8])
 {
     uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -235,7 +230,6 @@ __device__ __forceinline__ void channel_step(uint32_t wrow, uint32_t cf, int l, 
         lo[p] = x.x;
         hi[p] = x.y;
     }
-    float v[8];
     if (T == 1) {
         values_depth1(lo[0], l, *reinterpret_cast<float(*)[4]>(&v[0]));
         values_depth1(hi[0], l, *reinterpret_cast<float(*)[4]>(&v[4]));
@@ -243,6 +237,12 @@ __device__ __forceinline__ void channel_step(uint32_t wrow, uint32_t cf, int l, 
         values_depth<T>(lo, l, *reinterpret_cast<float(*)[4]>(&v[0]));
         values_depth<T>(hi, l, *reinterpret_cast<float(*)[4]>(&v[4]));
     }
+}
+
+// acc += coefficient * value for the 8 tokens x G heads of one channel.
+template <int G>
+__device__ __forceinline__ void channel_macs(const float (&v)[8], uint32_t cf, float2 (&acc)[8][head_pairs<G>()])
+{
     constexpr int GP = head_pairs<G>();
     float2 k[GP];
 #pragma unroll
@@ -260,14 +260,18 @@ __device__ __forceinline__ void channel_step(uint32_t wrow, uint32_t cf, int l, 
     }
 }
 
+// All channels of depth T in a chunk.
 template <int G, int T>
 __device__ __forceinline__ void depth_class(uint32_t& wrow, uint32_t& cf, int count, int l,
                                             float2 (&acc)[8][head_pairs<G>()])
 {
+    constexpr uint32_t kCf = kBlocksPerWarp * coef_pairs<G>() * 8;
     for (int i = 0; i < count; ++i) {
-        channel_step<G, T>(wrow, cf, l, acc);
+        float v[8];
+        channel_values<T>(wrow, l, v);
+        channel_macs<G>(v, cf, acc);
         wrow += T * kRowBytes;
-        cf += kBlocksPerWarp * coef_pairs<G>() * 8;
+        cf += kCf;
     }
 }
 
@@ -499,30 +503,40 @@ scan_kernel(const ScanArgs a)
                 }
             } else {
                 const int64_t ptile = ltile * a.tile_stride;
-                // Most lanes hold no survivor: a head's 8 scores are tested
-                // one by one only when their maximum reaches its threshold.
+                const bool whole = (ltile + 1) * kScanTileTokens <= a.n;   // no token of the tile is past n
+                int2* const ent_h = a.entries + h * G * a.cap;
+                auto keep = [&](int m, int g, float sv) {
+                    const int64_t i = tok0 + (m >> 2) * 32 + 8 * (m & 3);
+                    if (!whole && i >= a.n) return;
+                    const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
+                    if (S.direct[g]) {
+                        ent_h[g * a.cap + i] = ent;
+                    } else {
+                        const int p = atomicAdd(&S.tile_cnt[ti][g], 1);
+                        if (p < a.tslot) ent_h[g * a.cap + ptile * a.tslot + p] = ent;
+                    }
+                };
+                // Survivor mask over (head, token): one compare per score and
+                // no branch; then one pass per survivor, usually none.
+                using Mask = typename std::conditional<(G <= 4), uint32_t, unsigned long long>::type;
+                Mask mask = 0;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     const float tau = S.tau[g];
-                    const float mx = max3f(max3f(acc_at<G>(acc, 0, g), acc_at<G>(acc, 1, g), acc_at<G>(acc, 2, g)),
-                                           max3f(acc_at<G>(acc, 3, g), acc_at<G>(acc, 4, g), acc_at<G>(acc, 5, g)),
-                                           fmaxf(acc_at<G>(acc, 6, g), acc_at<G>(acc, 7, g)));
-                    if (mx >= tau) {
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) {
-                            const float sv = acc_at<G>(acc, m, g);
-                            const int64_t i = tok0 + (m >> 2) * 32 + 8 * (m & 3);
-                            if (sv >= tau && i < a.n) {
-                                const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
-                                if (S.direct[g]) {
-                                    a.entries[(h * G + g) * a.cap + i] = ent;
-                                } else {
-                                    const int p = atomicAdd(&S.tile_cnt[ti][g], 1);
-                                    if (p < a.tslot) a.entries[(h * G + g) * a.cap + ptile * a.tslot + p] = ent;
-                                }
-                            }
-                        }
-                    }
+                    for (int m = 0; m < 8; ++m) mask |= static_cast<Mask>(acc_at<G>(acc, m, g) >= tau) << (g * 8 + m);
+                }
+                while (mask) {
+                    const int bit = (G <= 4 ? __ffs(static_cast<uint32_t>(mask)) : __ffsll(static_cast<long long>(mask))) - 1;
+                    mask &= mask - 1;
+                    const int g = bit >> 3, m = bit & 7;
+                    float sv = 0.0f;
+#pragma unroll
+                    for (int gg = 0; gg < G; ++gg)
+#pragma unroll
+                        for (int mm = 0; mm < 8; ++mm)
+                            if (gg == g && mm == m) sv = acc_at<G>(acc, mm, gg);
+                    keep(m, g, sv);
                 }
             }
         }

@@ -187,6 +187,8 @@ def test_candidate_path_equals_dense(fathom_gpu, orc, budget):
     torch.cuda.synchronize()
     assert torch.all(c_cnt >= 0)   # every group proved exact without a rerun
     assert torch.equal(c_idx, d_idx) and torch.equal(c_uni, d_uni) and torch.equal(c_cnt, d_cnt)
+    # No ring wait of either scan gave up: the device fault word is clear.
+    assert fathom_gpu.device_status() == fathom_gpu.OK
 
 
 def test_candidate_overflow_is_flagged_and_repaired(fathom_gpu, orc):
