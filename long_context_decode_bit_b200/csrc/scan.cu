@@ -561,9 +561,15 @@ int launch_scan_g(ScanArgs a, int64_t ltiles, unsigned H, cudaStream_t stream)
     const cudaError_t e = cudaFuncSetAttribute(scan_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_status(e);
-    // Several tiles per CTA amortise the per-CTA plan set-up, as long as the
-    // grid still fills the GPU several times over.
-    int64_t per = ltiles * H / 1800;
+    // Several tiles per CTA amortise the per-CTA plan set-up: as many as
+    // keep the grid at two or more waves of resident CTAs (capped).
+#ifndef FATHOM_SCAN_WAVES
+#define FATHOM_SCAN_WAVES 2
+#endif
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t slots = static_cast<int64_t>(sms) * FATHOM_SCAN_MIN_CTAS * FATHOM_SCAN_WAVES;
+    const int64_t per = ceil_div(ltiles * static_cast<int64_t>(H), slots);
     a.tiles_per_cta = static_cast<int>(per < 1 ? 1 : (per > FATHOM_SCAN_TILES_CAP ? FATHOM_SCAN_TILES_CAP : per));
     const unsigned gx = static_cast<unsigned>(ceil_div(ltiles, a.tiles_per_cta));
     scan_kernel<G><<<dim3(gx, H), kScanThreads, smem, stream>>>(a);

@@ -10,8 +10,8 @@
 // lowest indices win (dense scores are scanned in index order; candidate
 // lists are unordered, so their ties are sorted by index).  The k winners
 // are then sorted by (score desc, index asc) with a shared-memory bitonic
-// sort on 64-bit composite keys.  A two-pass select on the top 16 key bits
-// picks the candidate threshold tau from the sample scores.
+// sort on 64-bit composite keys.  The same select, over per-thread maxima
+// of the sample scores, picks the candidate threshold tau.
 #include "common.cuh"
 
 namespace fathom {
@@ -110,64 +110,6 @@ __host__ __device__ inline int pow2_at_least(int x)
     return p;
 }
 
-// A sample of up to kTauRegs * 2 * blockDim.x scores is read from global
-// memory once and kept in registers as the top 16 bits of each order key,
-// two per register.  The select then runs on those 16 bits (11 + 5), and
-// tau is the smallest score whose key has the selected top 16 bits: never
-// above the exact m-th largest sample score, and within 2^-7 of it
-// relatively, so the candidate pass keeps at least as many keys as the
-// exact threshold would, and a few percent more at most.
-constexpr int kTauRegs = 16;
-
-__device__ uint32_t block_select16(const uint32_t (&pk)[kTauRegs], int count, int kk, uint32_t* hist, uint32_t* sh)
-{
-    uint32_t prefix = 0, mask = 0;
-#pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-        const int shift = pass == 0 ? 5 : 0;
-        const int width = pass == 0 ? 11 : 5;
-        const uint32_t dmask = (1u << width) - 1u;
-        const int nbins = 1 << width;
-        for (int b = threadIdx.x; b < kRadixBins; b += blockDim.x) hist[b] = 0;
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 2 * kTauRegs; ++j) {
-            const int i = static_cast<int>(threadIdx.x) + j * kTopkThreads;
-            const uint32_t key = (pk[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-            if (i < count && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            // Lane L owns the bins [top - per, top) (pass 2: lanes 0..31 one bin each).
-            const int lane = threadIdx.x, per = nbins >= 32 ? nbins / 32 : 1, top = nbins - per * lane;
-            uint32_t lsum = 0;
-            for (int b = top - 1; b >= top - per; --b) lsum += hist[b];
-            uint32_t incl = lsum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t v = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const uint32_t excl = incl - lsum;
-            const unsigned bal = __ballot_sync(kFull, excl < static_cast<uint32_t>(kk) &&
-                                                          static_cast<uint32_t>(kk) <= incl);
-            if (lane == __ffs(bal) - 1) {
-                uint32_t c = excl;
-                for (int b = top - 1; b >= top - per; --b) {
-                    if (c + hist[b] >= static_cast<uint32_t>(kk)) { sh[0] = b; sh[1] = c; break; }
-                    c += hist[b];
-                }
-            }
-        }
-        __syncthreads();
-        kk -= static_cast<int>(sh[1]);
-        prefix |= sh[0] << shift;
-        mask |= dmask << shift;
-        __syncthreads();
-    }
-    return prefix;   // top 16 bits of the kk-th largest key
-}
-
 // Header of a group's candidate buffer: the threshold, and the counters reset.
 __device__ __forceinline__ void write_header(CandHeader* hdr, int64_t hg, float tau, int64_t n_sample, int64_t n_keys)
 {
@@ -178,35 +120,39 @@ __device__ __forceinline__ void write_header(CandHeader* hdr, int64_t hg, float 
     hdr[hg].pad = 0;
 }
 
-// Threshold for the candidate pass, tau (see block_select16), of each head
-// whose sample fits in registers (or -inf without a sample); also resets the
-// candidate counters.
+// Threshold for the candidate pass (or -inf without a sample); also resets
+// the candidate counters.  Each thread takes the maximum of its share of the
+// sample scores, and tau is the m-th largest of those kTopkThreads maxima.
+// That is never above the m-th largest sample score (each thread gives at
+// most one of the top m), so the pass keeps at least as many keys as the
+// exact threshold would.  For m far below the thread count it is close:
+// m of the top sample scores land in different threads but for a few
+// collisions, and each collision only lowers tau to the next score.  The
+// sample is read from global memory once.
 __global__ void __launch_bounds__(kTopkThreads)
 tau_kernel(const float* __restrict__ sample, CandHeader* __restrict__ hdr, int64_t n_sample, int64_t m_rank,
            int64_t n_keys)
 {
     __shared__ uint32_t hist[kRadixBins];
+    __shared__ uint32_t tmax[kTopkThreads];
     __shared__ uint32_t sh[2];
     const int64_t hg = blockIdx.x;
     float tau = -INFINITY;
     if (n_sample > 0) {
         const float* s = sample + hg * n_sample;
-        const int ns = static_cast<int>(n_sample);   // at most 2 * kTauRegs * kTopkThreads here
-        uint32_t pk[kTauRegs];
-#pragma unroll
-        for (int j = 0; j < kTauRegs; ++j) {
-            const int i0 = static_cast<int>(threadIdx.x) + 2 * j * kTopkThreads, i1 = i0 + kTopkThreads;
-            const uint32_t k0 = i0 < ns ? order_key(s[i0]) >> 16 : 0u;
-            const uint32_t k1 = i1 < ns ? order_key(s[i1]) >> 16 : 0u;
-            pk[j] = k0 | (k1 << 16);
-        }
-        tau = key_to_float(block_select16(pk, ns, static_cast<int>(m_rank), hist, sh) << 16);
+        uint32_t mk = 0;   // order key of the thread's maximum (0: none, below every score's key)
+        for (int64_t i = threadIdx.x; i < n_sample; i += blockDim.x) mk = max(mk, order_key(s[i]));
+        tmax[threadIdx.x] = mk;
+        __syncthreads();
+        const Select r = block_select([&](int64_t i) { return tmax[i]; }, kTopkThreads, static_cast<int>(m_rank),
+                                      hist, sh);
+        tau = key_to_float(r.T);
     }
     if (threadIdx.x == 0) write_header(hdr, hg, tau, n_sample, n_keys);
 }
 
-// The same for samples too large for registers: the exact m-th largest
-// sample score, from three radix passes over global memory.
+// The same with the exact m-th largest sample score (three radix passes
+// over the sample), for m beyond a small fraction of the thread count.
 __global__ void __launch_bounds__(kTopkThreads)
 tau_kernel_large(const float* __restrict__ sample, CandHeader* __restrict__ hdr, int64_t n_sample, int64_t m_rank,
                  int64_t n_keys)
@@ -401,7 +347,7 @@ union_kernel(const int32_t* __restrict__ idx, int G, int k, int upow2, int32_t* 
 int launch_tau(const float* sample, CandHeader* hdr, int64_t heads, int64_t n_sample, int64_t m_rank,
                int64_t n_keys, cudaStream_t stream)
 {
-    if (n_sample > static_cast<int64_t>(2 * kTauRegs) * kTopkThreads)
+    if (n_sample > 0 && m_rank * 8 > kTopkThreads)
         tau_kernel_large<<<static_cast<unsigned>(heads), kTopkThreads, 0, stream>>>(sample, hdr, n_sample, m_rank,
                                                                                   n_keys);
     else
