@@ -50,6 +50,8 @@ def _lib():
         lib.orc_topk.argtypes = [P, I64, I, I64, I, P, P, P]
         lib.orc_dequant_rows.restype = I
         lib.orc_dequant_rows.argtypes = [P, P, I64, I, I64, I64, P, I64, P, I, P]
+        lib.orc_calibrate.restype = I
+        lib.orc_calibrate.argtypes = [P, I, I64, I64, I, I64, I64, P, P, P]
         _LIB = lib
     return _LIB
 
@@ -184,3 +186,24 @@ def dequant_rows(planes: np.ndarray, scales: np.ndarray, n: int, rows: np.ndarra
     _check(_lib().orc_dequant_rows(_ptr(planes), _ptr(scales), H, D, n, planes.shape[-1], _ptr(rows), M,
                                    None if rc is None else _ptr(rc), int(bits), _ptr(out)), "dequant_rows")
     return out
+
+
+def calibrate(keys: np.ndarray, n: int | None = None, with_cov: bool = True):
+    """fp64 (mean [H][D], population variance [H][D], covariance [H][D][D] or
+    None) of each group's first n keys; keys [H][n_total][D] float32 or
+    uint16 bf16 bit patterns."""
+    keys = np.ascontiguousarray(keys)
+    if keys.dtype == np.float32:
+        dt = 0
+    elif keys.dtype == np.uint16:
+        dt = 1
+    else:
+        raise TypeError("keys must be float32 or uint16 (bf16 bits)")
+    H, nt, D = keys.shape
+    n = nt if n is None else int(n)
+    mean = np.zeros((H, D), dtype=np.float64)
+    var = np.zeros((H, D), dtype=np.float64)
+    cov = np.zeros((H, D, D), dtype=np.float64) if with_cov else None
+    _check(_lib().orc_calibrate(_ptr(keys), dt, H, n, D, nt * D, D, _ptr(mean), _ptr(var),
+                                _ptr(cov) if with_cov else None), "calibrate")
+    return mean, var, cov

@@ -28,6 +28,11 @@
  *                      (byte-accounting section, top-k bullet)
  *   orc_dequant_rows   whole key rows rebuilt from the planes (limits
  *                      section, storage-overhead paragraph)
+ *   orc_calibrate      per-KV-head key statistics from the session's own
+ *                      keys: mean, population variance (the sigma^2 of the
+ *                      water-filling section) and covariance (experiments
+ *                      section, calibration-domain paragraph; rotated
+ *                      basis of the multi-model paragraph)
  */
 #include <math.h>
 #include <stdint.h>
@@ -409,5 +414,54 @@ int orc_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t H, 
             }
         }
     }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Key statistics of each group over its first n keys (experiments     */
+/* section: sigma^2 "measured once on calibration keys"; the session's */
+/* own prefill keys may serve, one covariance per KV head).  Two passes */
+/* in double: mean_j = (1/n) sum_i k_ij, then the centred population    */
+/* moments cov_ab = (1/n) sum_i (k_ia - mean_a)(k_ib - mean_b), whose   */
+/* diagonal is var_j.  mean and cov may be NULL; n = 0 gives zeros.     */
+/* ------------------------------------------------------------------ */
+int orc_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
+                  int64_t stride_h, int64_t stride_tok, double* mean, double* var, double* cov)
+{
+    if (!keys || !var || H < 0 || n < 0 || D <= 0) return ORC_EINVAL;
+    double* mu = (double*)calloc((size_t)D, sizeof(double));
+    double* row = (double*)calloc((size_t)D, sizeof(double));
+    if (!mu || !row) { free(mu); free(row); return ORC_ENOMEM; }
+    for (int64_t h = 0; h < H; ++h) {
+        for (int j = 0; j < D; ++j) mu[j] = 0.0;
+        for (int64_t i = 0; i < n; ++i)
+            for (int j = 0; j < D; ++j) {
+                int64_t off = h * stride_h + i * stride_tok + j;
+                mu[j] += key_dtype == 1 ? orc_bf16_value(((const uint16_t*)keys)[off]) : (double)((const float*)keys)[off];
+            }
+        for (int j = 0; j < D; ++j) mu[j] = n > 0 ? mu[j] / (double)n : 0.0;
+        double* c = cov ? cov + h * (int64_t)D * D : NULL;
+        if (c) for (int64_t e = 0; e < (int64_t)D * D; ++e) c[e] = 0.0;
+        for (int j = 0; j < D; ++j) var[h * D + j] = 0.0;
+        for (int64_t i = 0; i < n; ++i) {
+            for (int j = 0; j < D; ++j) {
+                int64_t off = h * stride_h + i * stride_tok + j;
+                double v = key_dtype == 1 ? orc_bf16_value(((const uint16_t*)keys)[off]) : (double)((const float*)keys)[off];
+                row[j] = v - mu[j];
+                var[h * D + j] += row[j] * row[j];
+            }
+            if (c)
+                for (int a = 0; a < D; ++a)
+                    for (int b = 0; b < D; ++b) c[(int64_t)a * D + b] += row[a] * row[b];
+        }
+        for (int j = 0; j < D; ++j) {
+            var[h * D + j] = n > 0 ? var[h * D + j] / (double)n : 0.0;
+            if (mean) mean[h * D + j] = mu[j];
+        }
+        if (c && n > 0)
+            for (int64_t e = 0; e < (int64_t)D * D; ++e) c[e] /= (double)n;
+    }
+    free(mu);
+    free(row);
     return ORC_OK;
 }

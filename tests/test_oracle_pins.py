@@ -476,3 +476,60 @@ def test_dequant_rows_is_the_midrise_value_of_each_key(orc):
                         continue
                     s = Fraction(orc.fp16_value(int(scales[h, j, i // 64])))
                     assert Fraction(out[h, r, j]) == midrise(Fraction(float(keys[h, i, j])), bits, s)
+
+
+# --------------------------------------------------------------------------
+# Session calibration statistics (section 方法二: sigma^2 measured on
+# calibration keys; experiments section: one covariance per KV head from
+# the session's own prefill keys)
+# --------------------------------------------------------------------------
+def test_calibrate_closed_forms(orc):
+    """Values the definitions fix: a constant channel has variance 0 and
+    its own value as mean; a +-a two-point channel has mean 0 and variance
+    a^2; two channels equal up to sign have covariance -+var."""
+    n = 512
+    k = np.zeros((1, n, 4), dtype=np.float32)
+    k[0, :, 0] = 3.25
+    k[0, ::2, 1], k[0, 1::2, 1] = 1.5, -1.5
+    k[0, :, 2] = (2 * np.arange(n) - (n - 1)) / 512.0        # evenly spaced, exact in fp32
+    k[0, :, 3] = -k[0, :, 2]
+    mean, var, cov = orc.calibrate(k)
+    assert mean[0, 0] == 3.25 and var[0, 0] == 0.0 and not np.any(cov[0, 0]) and not np.any(cov[0, :, 0])
+    assert mean[0, 1] == 0.0 and var[0, 1] == 2.25
+    v2 = var[0, 2]
+    # variance of i = 0..n-1 is (n^2 - 1)/12; the channel is (2i - (n-1))/512
+    assert v2 == pytest.approx(4.0 * (n * n - 1) / 12.0 / 512.0 ** 2, rel=1e-12)
+    assert cov[0, 2, 3] == pytest.approx(-v2, rel=1e-12) and cov[0, 3, 3] == pytest.approx(v2, rel=1e-12)
+
+
+def test_calibrate_matches_library_moments_and_invariances(orc):
+    """Against numpy's population variance and biased covariance (the
+    special case of library routines); shift leaves the centred moments
+    unchanged, scaling by a multiplies them by a^2; the covariance is
+    symmetric, positive semi-definite, with the variances on its diagonal;
+    bf16 keys give the statistics of their fp32 values; n selects a prefix."""
+    rng = np.random.default_rng(7)
+    H, nt, D = 3, 700, 16
+    std = np.exp(rng.normal(0, 1, D))
+    k = (rng.standard_normal((H, nt, D)) * std + rng.normal(0, 2, D)).astype(np.float32)
+    n = 600
+    mean, var, cov = orc.calibrate(k, n=n)
+    x = k[:, :n].astype(np.float64)
+    assert np.allclose(mean, x.mean(1), rtol=1e-12, atol=1e-12)
+    assert np.allclose(var, x.var(1), rtol=1e-10)
+    for h in range(H):
+        assert np.allclose(cov[h], np.cov(x[h].T, bias=True), rtol=1e-9, atol=1e-12)
+        assert np.array_equal(cov[h], cov[h].T)
+        assert np.linalg.eigvalsh(cov[h]).min() > -1e-9 * np.trace(cov[h])
+        assert np.allclose(np.diag(cov[h]), var[h], rtol=1e-12)
+    m2, v2, c2 = orc.calibrate((k + np.float32(4.0)).astype(np.float32), n=n)   # shift (exact in fp32 here? not always)
+    assert np.allclose(v2, var, rtol=1e-5) and np.allclose(m2, mean + 4.0, rtol=1e-6)
+    m3, v3, c3 = orc.calibrate((k * np.float32(2.0)).astype(np.float32), n=n)   # exact scaling by 2
+    assert np.allclose(v3, 4.0 * var, rtol=1e-12) and np.allclose(c3, 4.0 * cov, rtol=1e-12, atol=1e-12)
+    kb = (k.view(np.uint32) >> 16).astype(np.uint16)              # bf16 truncation of k
+    kf = (kb.astype(np.uint32) << 16).view(np.float32)            # ... and its exact fp32 value
+    mb, vb, cb = orc.calibrate(kb, n=n)
+    mf, vf, cf = orc.calibrate(np.ascontiguousarray(kf), n=n)
+    assert np.array_equal(mb, mf) and np.array_equal(vb, vf) and np.array_equal(cb, cf)
+    m0, v0, c0 = orc.calibrate(k, n=0)
+    assert not np.any(m0) and not np.any(v0) and not np.any(c0)
