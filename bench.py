@@ -543,6 +543,22 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     out["reconstruct_union_rows"] = {"ms": tot / 5, "rows": nrows, "rows_per_s": nrows / (tot / 5 / 1e3),
                                      "out_GBps": nrows * w.D * 4 / (tot / 5 / 1e3) / 1e9}
     del st, rows_out
+    # Session calibration from the session's own keys: one layer's 8 KV heads
+    # and one KV head at n = 100,000, with and without the covariance.
+    from long_context_decode_bit_b200 import inputs as _inputs
+    cw = dataclasses.replace(_inputs.STEP_1M, name="calibration-8x100000", H=8, n=100_000, seed=21)
+    ck = _inputs.keys(cw, 0, cw.H, device=device)
+    cws = torch.empty(fathom.calibrate_workspace_bytes(cw.H, cw.D, True), dtype=torch.uint8, device=device)
+    cal = {}
+    for label, kk, cov in (("layer_8_heads_cov", ck, True), ("layer_8_heads_sigma2", ck, False),
+                           ("one_head_cov", ck[:1], True)):
+        def calf(ev, kk=kk, cov=cov):
+            fathom.calibrate(kk, with_cov=cov, workspace=cws)
+        calf(None)
+        tot, _ = time_steps(calf, 5, 2, device)
+        cal[label] = {"ms": tot / 5, "heads": kk.shape[0], "n": cw.n}
+    out["calibrate_100k"] = cal
+    del ck, cws
     layers = w.H // 8 if w.H % 8 == 0 else 1
     per = w.H // layers
     steps = [fathom.Step(planes[l * per:(l + 1) * per], scales[l * per:(l + 1) * per], w.n,

@@ -117,6 +117,42 @@ int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
                 fathom_stream_t stream);
 
 /*
+ * fathom_calibrate_workspace_bytes -- scratch fathom_calibrate needs (HOST
+ * call); 0 for unsupported sizes.
+ */
+size_t fathom_calibrate_workspace_bytes(int64_t H, int D, int with_cov);
+
+/*
+ * fathom_calibrate -- per-group key statistics over the first n keys: the
+ * channel variance sigma^2 that fathom_plan takes (方法二: measured once on
+ * calibration keys), and optionally the mean and the covariance from which
+ * a caller builds a rotated basis (实验 section: statistics from the
+ * session's own prefill keys, one covariance per KV head).
+ *
+ *   mean_j  = (1/n) sum_i k_ij
+ *   sigma2_j = (1/n) sum_i (k_ij - mean_j)^2            (population variance)
+ *   cov_ab  = (1/n) sum_i (k_ia - mean_a)(k_ib - mean_b)
+ *
+ * Sums run in double precision over k - k_0 (the group's first key) and are
+ * rounded once to fp32; the double atomics that combine chunks make the
+ * last fp64 bits depend on timing, so an output can differ between runs
+ * only where its fp64 value lies next to an fp32 rounding boundary.
+ *
+ *   keys        DEVICE, [H][n][D] as for fathom_pack (fp32 or bf16, strides in
+ *               elements); not read when n == 0.
+ *   mean        DEVICE out (may be NULL), fp32 [H][D].
+ *   sigma2      DEVICE out, fp32 [H][D].
+ *   cov         DEVICE out (may be NULL), fp32 [H][D][D].
+ *   workspace, ws_bytes  DEVICE scratch of at least
+ *               fathom_calibrate_workspace_bytes(H, D, cov != NULL) bytes,
+ *               256-byte aligned (FATHOM_ERR_WORKSPACE if smaller).
+ * n == 0 gives zeros.  D as for fathom_pack; H <= 65535.
+ */
+int fathom_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
+                     int64_t key_stride_h, int64_t key_stride_tok, float* mean, float* sigma2,
+                     float* cov, void* workspace, size_t ws_bytes, fathom_stream_t stream);
+
+/*
  * fathom_plan -- per-group reverse water-filling (方法二).
  *
  * Channel importance, in single precision with round-to-nearest and in this

@@ -22,6 +22,10 @@ int launch_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t 
                         int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count, int bits,
                         float* out, cudaStream_t stream);
 
+size_t calibrate_workspace_bytes(int64_t H, int D, bool with_cov);
+int launch_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t sh, int64_t st,
+                     float* mean, float* sigma2, float* cov, void* ws, cudaStream_t stream);
+
 static thread_local int g_last_cuda_error = 0;
 
 int cuda_status(cudaError_t e)
@@ -115,6 +119,36 @@ int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, in
     FATHOM_TRY(check_device_ptr(scales));
     return launch_pack(keys, key_dtype, H, n, D, key_stride_h, key_stride_tok, planes, scales, nb_stride,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fathom_calibrate_workspace_bytes(int64_t H, int D, int with_cov)
+{
+    if (H <= 0 || !dims_ok(D, 1)) return 0;
+    return calibrate_workspace_bytes(H, D, with_cov != 0);
+}
+
+int fathom_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t key_stride_h,
+                     int64_t key_stride_tok, float* mean, float* sigma2, float* cov, void* workspace, size_t ws_bytes,
+                     fathom_stream_t stream)
+{
+    if (H < 0 || n < 0 || n >= (1LL << 40)) return FATHOM_ERR_INVALID_ARG;
+    if (key_dtype != FATHOM_KEYS_F32 && key_dtype != FATHOM_KEYS_BF16) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
+    if (H == 0) return FATHOM_OK;
+    if (H > 65535) return FATHOM_ERR_UNSUPPORTED;
+    if (key_stride_tok < D || (H > 1 && key_stride_h < n * key_stride_tok)) return FATHOM_ERR_INVALID_ARG;
+    if (!sigma2) return FATHOM_ERR_INVALID_ARG;
+    if (ws_bytes < calibrate_workspace_bytes(H, D, cov != nullptr)) return FATHOM_ERR_WORKSPACE;
+    if (!aligned(keys, key_dtype == FATHOM_KEYS_F32 ? 4 : 2) || !aligned(sigma2, 4) || (mean && !aligned(mean, 4)) ||
+        (cov && !aligned(cov, 4)) || !aligned(workspace, 256))
+        return FATHOM_ERR_UNSUPPORTED;
+    if (n > 0) FATHOM_TRY(check_device_ptr(keys));
+    FATHOM_TRY(check_device_ptr(sigma2));
+    FATHOM_TRY(check_device_ptr(workspace));
+    if (mean) FATHOM_TRY(check_device_ptr(mean));
+    if (cov) FATHOM_TRY(check_device_ptr(cov));
+    return launch_calibrate(keys, key_dtype, H, n, D, key_stride_h, key_stride_tok, mean, sigma2, cov, workspace,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,

@@ -36,7 +36,7 @@ EXPORTS = (
     "fathom_version", "fathom_status_string", "fathom_last_cuda_error", "fathom_nb_stride",
     "fathom_pack", "fathom_plan", "fathom_plan_fixed", "fathom_scan_cand_bytes", "fathom_scan",
     "fathom_topk_workspace_bytes", "fathom_topk", "fathom_dequant_rows", "fathom_scan_topk_noalloc",
-    "fathom_device_status",
+    "fathom_device_status", "fathom_calibrate_workspace_bytes", "fathom_calibrate",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -80,6 +80,8 @@ def load(path: str | None = None):
         "fathom_dequant_rows": (I, [P, P, I64, I, I64, I64, P, I64, P, I, P, P]),
         "fathom_scan_topk_noalloc": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, P, P]),
         "fathom_device_status": (I, [I, P]),
+        "fathom_calibrate_workspace_bytes": (SZ, [I64, I, I]),
+        "fathom_calibrate": (I, [P, I, I64, I64, I, I64, I64, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -255,6 +257,37 @@ def scan_topk_noalloc(planes, scales, n: int, active, n_active, q, k: int, out=N
                                           _p(n_active), _p(q), G, int(k), _p(idx), _p(uni), _p(cnt),
                                           _stream(stream)), "fathom_scan_topk_noalloc")
     return idx, uni, cnt
+
+
+def calibrate_workspace_bytes(H: int, D: int, with_cov: bool) -> int:
+    return int(lib().fathom_calibrate_workspace_bytes(H, D, 1 if with_cov else 0))
+
+
+def calibrate(keys: torch.Tensor, n: int | None = None, with_mean: bool = True, with_cov: bool = False,
+              workspace=None, stream=None):
+    """Per-group key statistics over the first ``n`` keys of keys [H][n_total][D]
+    (fp32 or bf16): (mean [H][D] or None, sigma2 [H][D], cov [H][D][D] or None),
+    all fp32."""
+    H, nt, D = keys.shape
+    n = nt if n is None else int(n)
+    if keys.dtype == torch.float32:
+        dt = KEYS_F32
+    elif keys.dtype == torch.bfloat16:
+        dt = KEYS_BF16
+    else:
+        raise TypeError("keys must be float32 or bfloat16")
+    if keys.stride(2) != 1:
+        raise ValueError("keys must be contiguous along D")
+    dev = keys.device
+    sigma2 = torch.empty((H, D), dtype=torch.float32, device=dev)
+    mean = torch.empty((H, D), dtype=torch.float32, device=dev) if with_mean else None
+    cov = torch.empty((H, D, D), dtype=torch.float32, device=dev) if with_cov else None
+    need = calibrate_workspace_bytes(H, D, with_cov)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check(lib().fathom_calibrate(_p(keys), dt, H, n, D, keys.stride(0), keys.stride(1), _p(mean), _p(sigma2),
+                                  _p(cov), _p(workspace), workspace.numel(), _stream(stream)), "fathom_calibrate")
+    return mean, sigma2, cov
 
 
 def device_status(clear: bool = False, stream=None) -> int:

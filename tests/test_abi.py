@@ -54,6 +54,12 @@ def test_host_only_entry_points(lib):
     # spread over the tiles + one count per tile + 32768 sample scores of 4 B)
     per_head = 16384 * 8 + 32768 * 4
     assert 1152 * per_head <= big < 1152 * (per_head + 4096 + 16) + 4 * 256
+    # calibration scratch: two fp64 sums per (group, channel), plus the
+    # fp64 D x D sums with the covariance
+    assert lib.fathom_calibrate_workspace_bytes(0, 128, 0) == 0
+    assert lib.fathom_calibrate_workspace_bytes(8, 100, 0) == 0              # unsupported D
+    assert lib.fathom_calibrate_workspace_bytes(8, 128, 0) == 2 * 8 * 128 * 8
+    assert lib.fathom_calibrate_workspace_bytes(8, 128, 1) == 2 * 8 * 128 * 8 + 8 * 128 * 128 * 8
 
 
 def test_rejections_before_any_cuda_call(lib):
@@ -72,6 +78,12 @@ def test_rejections_before_any_cuda_call(lib):
     assert lib.fathom_scan(n, n, 1, 100, 100, 2, n, n, n, 4, 0, n, n, 0, 1, n) == fathom.ERR_UNSUPPORTED
     assert lib.fathom_topk(n, n, 1, 4, 100, 5, n, n, n, n, 0, n) == fathom.ERR_INVALID_ARG   # neither input
     assert lib.fathom_topk(n, n, 1, 0, 100, 5, n, n, n, n, 0, n) == fathom.ERR_UNSUPPORTED   # G = 0
+    assert lib.fathom_calibrate(n, 3, 1, 64, 128, 64 * 128, 128, n, n, n, n, 0, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_calibrate(n, 0, 1, 64, 48, 64 * 48, 48, n, n, n, n, 0, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_calibrate(n, 0, 0, 64, 128, 0, 128, n, n, n, n, 0, n) == fathom.OK     # nothing to do
+    fake = ctypes.c_void_p(256)   # never dereferenced: the size check comes first
+    assert lib.fathom_calibrate(fake, 0, 2, 64, 128, 64 * 128, 128, n, fake, n, fake, 100, n) == fathom.ERR_WORKSPACE
+    assert lib.fathom_calibrate(fake, 0, 2, 64, 128, 64 * 128, 128, n, n, n, fake, 1 << 20, n) == fathom.ERR_INVALID_ARG
 
 
 def test_missing_library_fails_loudly(tmp_path):

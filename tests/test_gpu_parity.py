@@ -294,3 +294,44 @@ def test_append_repacks_the_tail_block(fathom_gpu, orc):
     assert torch.equal(planes, full_p) and torch.equal(scales, full_s)
     p_ref, s_ref = orc.pack(keys_for_oracle(k[:, :n]), nb_stride=nbs)
     assert np.array_equal(np_u64(planes), p_ref) and np.array_equal(np_u16(scales), s_ref)
+
+
+# --------------------------------------------------------------------------
+# Session calibration statistics (方法二 sigma^2; experiments section: one
+# covariance per KV head from the session's own prefill keys)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("w,n", [(inputs.TINY, None), (inputs.TINY, 1024),
+                                 (dataclasses.replace(inputs.LAYER_32K, name="cal", H=3, n=9000, seed=12), None),
+                                 (dataclasses.replace(inputs.TINY, name="cal-d64", H=2, D=64, n=777, seed=13), None),
+                                 (dataclasses.replace(inputs.STEP_1M_LLAMA, name="cal-corr", H=2, n=5000, seed=14), None)],
+                         ids=["tiny", "tiny-first-1024", "qk-bf16-9000", "d64-ragged", "corr-bf16-5000"])
+def test_calibrate_matches_oracle(fathom_gpu, orc, w, n):
+    """Mean and sigma^2 equal the oracle's fp64 values rounded to fp32 (a
+    one-ulp allowance covers the fp64 summation order); the covariance is
+    within fp32 rounding of the oracle's plus 1e-12 of sqrt(var_a var_b)."""
+    k = inputs.keys(w, 0, w.H, device=DEV)
+    mean, s2, cov = fathom_gpu.calibrate(k, n=n, with_cov=True)
+    torch.cuda.synchronize()
+    om, ov, oc = orc.calibrate(keys_for_oracle(k), n=n)
+    ulp = lambda x: np.spacing(np.abs(x).astype(np.float32)).astype(np.float64)
+    for got, ref in ((mean, om), (s2, ov)):
+        g = got.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(g - ref) <= ulp(ref) + 1e-30), np.abs(g - ref).max()
+    g = cov.cpu().numpy().astype(np.float64)
+    scale = np.sqrt(np.einsum("ha,hb->hab", ov, ov))
+    assert np.all(np.abs(g - oc) <= ulp(oc) + 1e-12 * scale + 1e-30)
+
+
+def test_calibrate_sigma2_feeds_the_plan(fathom_gpu, orc):
+    """sigma^2 from the calibration call over the first n_cal keys gives the
+    same plan as the harness statistic, bit for bit."""
+    w = inputs.LAYER_32K
+    k, q, s2 = make(w)
+    _, s2_gpu, _ = fathom_gpu.calibrate(k, n=w.n_cal, with_mean=False)
+    d_ref, a_ref, n_ref, _ = fathom_gpu.plan(s2, q, 48)
+    d_cal, a_cal, n_cal, _ = fathom_gpu.plan(s2_gpu, q, 48)
+    torch.cuda.synchronize()
+    diff = (s2_gpu != s2).sum().item()
+    assert diff <= 2   # one-ulp fp64 summation-order cases at most
+    if diff == 0:
+        assert torch.equal(d_ref, d_cal) and torch.equal(a_ref, a_cal) and torch.equal(n_ref, n_cal)
