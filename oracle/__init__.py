@@ -52,6 +52,8 @@ def _lib():
         lib.orc_dequant_rows.argtypes = [P, P, I64, I, I64, I64, P, I64, P, I, P]
         lib.orc_calibrate.restype = I
         lib.orc_calibrate.argtypes = [P, I, I64, I64, I, I64, I64, P, P, P]
+        lib.orc_union_attention.restype = I
+        lib.orc_union_attention.argtypes = [P, P, I, I64, I64, I, I64, I64, P, I, P, P, I64, ctypes.c_double, P]
         _LIB = lib
     return _LIB
 
@@ -207,3 +209,25 @@ def calibrate(keys: np.ndarray, n: int | None = None, with_cov: bool = True):
     _check(_lib().orc_calibrate(_ptr(keys), dt, H, n, D, nt * D, D, _ptr(mean), _ptr(var),
                                 _ptr(cov) if with_cov else None), "calibrate")
     return mean, var, cov
+
+
+def union_attention(k: np.ndarray, v: np.ndarray, q: np.ndarray, uni: np.ndarray, count: np.ndarray,
+                    scale: float | None = None):
+    """fp64 softmax attention [H][G][D] of each query head over its group's
+    union rows; k, v [H][n][D] float32 or uint16 bf16 bits (same dtype)."""
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    if k.dtype != v.dtype or k.shape != v.shape:
+        raise TypeError("k and v must share dtype and shape")
+    dt = {np.dtype(np.float32): 0, np.dtype(np.uint16): 1}[k.dtype]
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    uni = np.ascontiguousarray(uni, dtype=np.int32)
+    count = np.ascontiguousarray(count, dtype=np.int32)
+    H, n, D = k.shape
+    G = q.shape[1]
+    M = uni.shape[1]
+    sc = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    out = np.zeros((H, G, D), dtype=np.float64)
+    _check(_lib().orc_union_attention(_ptr(k), _ptr(v), dt, H, n, D, n * D, D, _ptr(q), G, _ptr(uni), _ptr(count),
+                                      M, sc, _ptr(out)), "union_attention")
+    return out

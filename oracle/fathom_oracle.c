@@ -33,6 +33,9 @@
  *                      water-filling section) and covariance (experiments
  *                      section, calibration-domain paragraph; rotated
  *                      basis of the multi-model paragraph)
+ *   orc_union_attention  softmax attention of each query head over its KV
+ *                      head's union of winner rows (byte-accounting
+ *                      section: the winner rows a step fetches)
  */
 #include <math.h>
 #include <stdint.h>
@@ -463,5 +466,61 @@ int orc_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
     }
     free(mu);
     free(row);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Attention over the union of winners (byte-accounting section: each    */
+/* step fetches the KV rows of the union of the G heads' top-k, at most  */
+/* G*k rows per KV head).  For group h, head g and the rows i in         */
+/* union[h][0 .. count_h):                                               */
+/*   s_i = scale * q_g . K_i,  p_i = exp(s_i - max s) / sum exp(s - max), */
+/*   out_g = sum_i p_i V_i.                                              */
+/* A count <= 0 (no rows, or an error status) gives a zero output.       */
+/* K and V: [H][n][D] with the given strides, fp32 or bf16 bits.         */
+/* ------------------------------------------------------------------ */
+int orc_union_attention(const void* kc, const void* vc, int kv_dtype, int64_t H, int64_t n, int D,
+                        int64_t stride_h, int64_t stride_tok, const float* q, int G, const int32_t* uni,
+                        const int32_t* count, int64_t M, double scale, double* out)
+{
+    if (!kc || !vc || !q || !uni || !count || !out || H < 0 || n < 0 || D <= 0 || G <= 0 || M < 0) return ORC_EINVAL;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)(M > 0 ? M : 1));
+    if (!sc) return ORC_ENOMEM;
+    for (int64_t h = 0; h < H; ++h) {
+        int64_t c = count[h] < 0 ? 0 : (count[h] > M ? M : count[h]);
+        for (int g = 0; g < G; ++g) {
+            const float* qg = q + (h * G + g) * (int64_t)D;
+            double* o = out + (h * G + g) * (int64_t)D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (c == 0) continue;
+            double mx = -INFINITY;
+            for (int64_t r = 0; r < c; ++r) {
+                int64_t i = uni[h * M + r];
+                if (i < 0 || i >= n) { free(sc); return ORC_EINVAL; }
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    int64_t off = h * stride_h + i * stride_tok + d;
+                    double kv = kv_dtype == 1 ? orc_bf16_value(((const uint16_t*)kc)[off]) : (double)((const float*)kc)[off];
+                    dot += (double)qg[d] * kv;
+                }
+                sc[r] = scale * dot;
+                if (sc[r] > mx) mx = sc[r];
+            }
+            double den = 0.0;
+            for (int64_t r = 0; r < c; ++r) {
+                sc[r] = exp(sc[r] - mx);
+                den += sc[r];
+            }
+            for (int64_t r = 0; r < c; ++r) {
+                int64_t i = uni[h * M + r];
+                for (int d = 0; d < D; ++d) {
+                    int64_t off = h * stride_h + i * stride_tok + d;
+                    double vv = kv_dtype == 1 ? orc_bf16_value(((const uint16_t*)vc)[off]) : (double)((const float*)vc)[off];
+                    o[d] += sc[r] / den * vv;
+                }
+            }
+        }
+    }
+    free(sc);
     return ORC_OK;
 }

@@ -533,3 +533,47 @@ def test_calibrate_matches_library_moments_and_invariances(orc):
     assert np.array_equal(mb, mf) and np.array_equal(vb, vf) and np.array_equal(cb, cf)
     m0, v0, c0 = orc.calibrate(k, n=0)
     assert not np.any(m0) and not np.any(v0) and not np.any(c0)
+
+
+# --------------------------------------------------------------------------
+# Attention over the union of winners (byte-accounting section: the rows a
+# step fetches are the union of the G heads' top-k)
+# --------------------------------------------------------------------------
+def test_union_attention_special_cases(orc):
+    """With every row in the union it is dense softmax attention (numpy
+    matmul + exp); one row returns that value row; a zero query averages the
+    union's value rows; the order of the union list does not matter; an
+    empty or error count gives zeros; bf16 K/V give the result of their
+    fp32 values."""
+    rng = np.random.default_rng(11)
+    H, n, D, G = 2, 300, 32, 4
+    k = rng.standard_normal((H, n, D)).astype(np.float32)
+    v = rng.standard_normal((H, n, D)).astype(np.float32)
+    q = rng.standard_normal((H, G, D)).astype(np.float32)
+    full = np.tile(np.arange(n, dtype=np.int32), (H, 1))
+    out = orc.union_attention(k, v, q, full, np.full(H, n, np.int32))
+    s = np.einsum("hgd,hnd->hgn", q.astype(np.float64), k.astype(np.float64)) / np.sqrt(D)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    assert np.allclose(out, np.einsum("hgn,hnd->hgd", p, v.astype(np.float64)), rtol=1e-12, atol=1e-13)
+    one = orc.union_attention(k, v, q, np.array([[17], [250]], np.int32), np.array([1, 1], np.int32))
+    assert np.array_equal(one[0], np.tile(v[0, 17].astype(np.float64), (G, 1)))
+    assert np.array_equal(one[1], np.tile(v[1, 250].astype(np.float64), (G, 1)))
+    rows = np.stack([rng.choice(n, 40, replace=False) for _ in range(H)]).astype(np.int32)
+    zq = np.zeros_like(q)
+    avg = orc.union_attention(k, v, zq, rows, np.full(H, 40, np.int32))
+    for h in range(H):
+        assert np.allclose(avg[h], np.tile(v[h, rows[h]].astype(np.float64).mean(0), (G, 1)), rtol=1e-12, atol=1e-14)
+    a = orc.union_attention(k, v, q, rows, np.full(H, 40, np.int32))
+    b = orc.union_attention(k, v, q, rows[:, ::-1].copy(), np.full(H, 40, np.int32))
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
+    pad = np.concatenate([rows, np.full((H, 10), -1, np.int32)], axis=1)   # -1 padded past the count
+    assert np.array_equal(orc.union_attention(k, v, q, pad, np.full(H, 40, np.int32)), a)
+    assert not np.any(orc.union_attention(k, v, q, pad, np.array([0, -6], np.int32)))
+    kb = (k.view(np.uint32) >> 16).astype(np.uint16)
+    vb = (v.view(np.uint32) >> 16).astype(np.uint16)
+    kf = (kb.astype(np.uint32) << 16).view(np.float32)
+    vf = (vb.astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(orc.union_attention(kb, vb, q, rows, np.full(H, 40, np.int32)),
+                          orc.union_attention(np.ascontiguousarray(kf), np.ascontiguousarray(vf), q, rows,
+                                              np.full(H, 40, np.int32)))
