@@ -542,7 +542,27 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     nrows = int(cnt.clamp(min=0).sum().item())
     out["reconstruct_union_rows"] = {"ms": tot / 5, "rows": nrows, "rows_per_s": nrows / (tot / 5 / 1e3),
                                      "out_GBps": nrows * w.D * 4 / (tot / 5 / 1e3) / 1e9}
-    del st, rows_out
+    # Attention of the step's query heads over their union rows, for the
+    # first layer's 8 groups (their full-precision K/V cache regenerated).
+    from long_context_decode_bit_b200 import inputs as _inp
+    la = min(8, w.H)
+    kc = _inp.keys(w, 0, la, device=device)
+    vc = _inp.values(w, 0, la, device=device)
+    uni8, cnt8 = uni[:la].contiguous(), cnt[:la].contiguous()
+    q8 = q[:la].float().contiguous()
+    att_out = torch.empty((la, w.G, w.D), dtype=torch.float32, device=device)
+    att_ws = torch.empty(fathom.union_attention_workspace_bytes(la, w.G, w.D, uni8.shape[1]), dtype=torch.uint8,
+                         device=device)
+
+    def att(ev):
+        fathom.union_attention(kc, vc, q8, uni8, cnt8, out=att_out, workspace=att_ws)
+    att(None)
+    tot, _ = time_steps(att, 5, 2, device)
+    arows = int(cnt8.clamp(min=0).sum().item())
+    out["union_attention_one_layer"] = {"groups": la, "ms": tot / 5, "rows": arows,
+                                        "kv_bytes": arows * 2 * w.D * kc.element_size(),
+                                        "kv_GBps": arows * 2 * w.D * kc.element_size() / (tot / 5 / 1e3) / 1e9}
+    del st, rows_out, kc, vc, att_out, att_ws
     # Session calibration from the session's own keys: one layer's 8 KV heads
     # and one KV head at n = 100,000, with and without the covariance.
     from long_context_decode_bit_b200 import inputs as _inputs

@@ -319,6 +319,40 @@ int fathom_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t 
                         int bits, float* out, fathom_stream_t stream);
 
 /*
+ * fathom_union_attention_workspace_bytes -- scratch fathom_union_attention
+ * needs (HOST call); 0 for unsupported sizes.
+ */
+size_t fathom_union_attention_workspace_bytes(int64_t H, int G, int D, int64_t M);
+
+/*
+ * fathom_union_attention -- the step after the scan: each query head's
+ * softmax attention over the KV rows of its group's union of winners (先算
+ * 一笔字节账, top-k bullet: a step fetches the union of the G heads'
+ * winner rows, at most G*k per KV head).  For group h, head g and the rows
+ * i = union_idx[h*M + r], r < union_count[h]:
+ *   s_i = scale * q_g . K_i,   out_g = sum_i softmax(s)_i V_i.
+ * fp32 arithmetic (expf); rows are taken in chunks of 256 and the chunks
+ * combined by their maxima (split over the union).  A union_count <= 0
+ * (none, or an error status from fathom_topk) gives a zero output; an
+ * index outside [0, n) is skipped.
+ *
+ *   k_cache, v_cache  DEVICE, [H][n][D] fp32 or bf16 (kv_dtype), the
+ *               session's full-precision cache, strides in elements.
+ *   q           DEVICE, fp32 [H][G][D].
+ *   union_idx, union_count  DEVICE, as fathom_topk writes them (M = G*k).
+ *   scale       usually 1/sqrt(D).
+ *   out         DEVICE out, fp32 [H][G][D].
+ *   workspace, ws_bytes  DEVICE scratch of at least
+ *               fathom_union_attention_workspace_bytes(H, G, D, M) bytes,
+ *               256-byte aligned.
+ * 1 <= M <= 65536; D, G as for fathom_plan; H <= 65535.
+ */
+int fathom_union_attention(const void* k_cache, const void* v_cache, int kv_dtype, int64_t H, int64_t n,
+                           int D, int64_t kv_stride_h, int64_t kv_stride_tok, const float* q, int G,
+                           const int32_t* union_idx, const int32_t* union_count, int64_t M, float scale,
+                           float* out, void* workspace, size_t ws_bytes, fathom_stream_t stream);
+
+/*
  * fathom_scan_topk_noalloc -- fathom_scan in CANDIDATE mode followed by
  * fathom_topk, for callers that cannot allocate device memory.  (The paper
  * has no counterpart: this is a deployment convenience of this library.)

@@ -26,6 +26,11 @@ size_t calibrate_workspace_bytes(int64_t H, int D, bool with_cov);
 int launch_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t sh, int64_t st,
                      float* mean, float* sigma2, float* cov, void* ws, cudaStream_t stream);
 
+size_t union_attention_workspace_bytes(int64_t H, int G, int D, int64_t M);
+int launch_union_attention(const void* k, const void* v, int kv_dtype, int64_t H, int64_t n, int D, int64_t sh,
+                           int64_t st, const float* q, int G, const int32_t* uni, const int32_t* count, int64_t M,
+                           float scale, float* out, void* ws, cudaStream_t stream);
+
 static thread_local int g_last_cuda_error = 0;
 
 int cuda_status(cudaError_t e)
@@ -149,6 +154,40 @@ int fathom_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int 
     if (cov) FATHOM_TRY(check_device_ptr(cov));
     return launch_calibrate(keys, key_dtype, H, n, D, key_stride_h, key_stride_tok, mean, sigma2, cov, workspace,
                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fathom_union_attention_workspace_bytes(int64_t H, int G, int D, int64_t M)
+{
+    if (H <= 0 || M < 1 || M > 65536 || !dims_ok(D, G)) return 0;
+    return union_attention_workspace_bytes(H, G, D, M);
+}
+
+int fathom_union_attention(const void* k_cache, const void* v_cache, int kv_dtype, int64_t H, int64_t n, int D,
+                           int64_t kv_stride_h, int64_t kv_stride_tok, const float* q, int G, const int32_t* union_idx,
+                           const int32_t* union_count, int64_t M, float scale, float* out, void* workspace,
+                           size_t ws_bytes, fathom_stream_t stream)
+{
+    if (H < 0 || n < 0 || n >= (1LL << 31) || M < 1 || M > 65536) return FATHOM_ERR_INVALID_ARG;
+    if (kv_dtype != FATHOM_KEYS_F32 && kv_dtype != FATHOM_KEYS_BF16) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
+    if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return FATHOM_ERR_INVALID_ARG;
+    if (H == 0) return FATHOM_OK;
+    if (H > 65535) return FATHOM_ERR_UNSUPPORTED;
+    if (kv_stride_tok < D || (H > 1 && kv_stride_h < n * kv_stride_tok)) return FATHOM_ERR_INVALID_ARG;
+    if (ws_bytes < union_attention_workspace_bytes(H, G, D, M)) return FATHOM_ERR_WORKSPACE;
+    const size_t ea = kv_dtype == FATHOM_KEYS_F32 ? 4 : 2;
+    if (!aligned(k_cache, ea) || !aligned(v_cache, ea) || !aligned(q, 4) || !aligned(union_idx, 4) ||
+        !aligned(union_count, 4) || !aligned(out, 4) || !aligned(workspace, 256))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(k_cache));
+    FATHOM_TRY(check_device_ptr(v_cache));
+    FATHOM_TRY(check_device_ptr(q));
+    FATHOM_TRY(check_device_ptr(union_idx));
+    FATHOM_TRY(check_device_ptr(union_count));
+    FATHOM_TRY(check_device_ptr(out));
+    FATHOM_TRY(check_device_ptr(workspace));
+    return launch_union_attention(k_cache, v_cache, kv_dtype, H, n, D, kv_stride_h, kv_stride_tok, q, G, union_idx,
+                                  union_count, M, scale, out, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,

@@ -1,0 +1,244 @@
+// fathom_union_attention: softmax attention of each query head over the
+// union of its KV head's winners.
+//
+// A decode step fetches the KV rows of the union of the G heads' top-k (at
+// most G*k rows per KV head; Fathom, byte-accounting section) and attends
+// over them.  For group h, head g and union rows i:
+//   s_i = scale * q_g . K_i,   out_g = sum_i softmax(s)_i V_i.
+// K and V are the session's full-precision cache, [H][n][D] (fp32 or bf16).
+//
+// Layout (split over the union, as in split-K decoding): a CTA takes a
+// chunk of up to kAttRows union rows of one group.
+//   1. Warp w scores rows w, w+8, ...: lane l reads channels l, l+32, ...
+//      of the row (64-byte coalesced pieces), keeps G partial dots and
+//      reduces them across the warp with butterfly shuffles.
+//   2. Warp g turns head g's chunk scores into exp(s - m_g) and their sum.
+//   3. Thread t accumulates channel t % D over the rows of its slice
+//      (t / D) for all G heads; the slices are summed in shared memory.
+// Each chunk leaves (m_g, l_g, o_g) in the workspace; the combine kernel
+// rescales them by exp(m_chunk - m_max) and divides by the total weight.
+// Everything is fp32 (expf, one rounding per operation).
+#include "common.cuh"
+
+namespace fathom {
+
+namespace {
+
+constexpr int kAttRows = 256;
+constexpr int kAttThreads = 256;
+constexpr unsigned kFullMask = 0xffffffffu;
+
+struct AttArgs {
+    const void* k;
+    const void* v;
+    int64_t n, sh, st, M;
+    int D;
+    const float* q;
+    const int32_t* uni;
+    const int32_t* count;
+    float scale;
+    int chunks;
+    float* pm;   // [H][chunks][G] chunk maxima
+    float* pl;   // [H][chunks][G] chunk weight sums
+    float* po;   // [H][chunks][G][D] chunk outputs (unnormalised)
+    float* out;  // [H][G][D]
+};
+
+template <int DT>
+__device__ __forceinline__ float kv_at(const void* p, int64_t off)
+{
+    if (DT == FATHOM_KEYS_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[off]);
+    return static_cast<const float*>(p)[off];
+}
+
+template <int DT, int G>
+__global__ void __launch_bounds__(kAttThreads)
+attend_chunk_kernel(const AttArgs a)
+{
+    extern __shared__ __align__(16) float sm[];
+    const int D = a.D;
+    float* qs = sm;                           // [G][D], scaled
+    float* sc = qs + G * D;                   // [G][kAttRows]: scores, then weights
+    float* red = sc + G * kAttRows;           // [slices][G][D]
+    int* rowi = reinterpret_cast<int*>(red + (kAttThreads / D) * G * D);   // [kAttRows]
+
+    const int64_t h = blockIdx.y;
+    const int c = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t cnt = min(max(static_cast<int64_t>(a.count[h]), int64_t{0}), a.M);
+    const int64_t r0 = static_cast<int64_t>(c) * kAttRows;
+    const int rows = static_cast<int>(max(int64_t{0}, min(static_cast<int64_t>(kAttRows), cnt - r0)));
+    const int64_t pbase = (h * a.chunks + c) * G;
+
+    for (int e = tid; e < G * D; e += kAttThreads) qs[e] = a.q[h * G * D + e] * a.scale;
+    for (int r = tid; r < rows; r += kAttThreads) {
+        const int32_t i = a.uni[h * a.M + r0 + r];
+        rowi[r] = (i >= 0 && i < a.n) ? i : -1;   // an index outside the cache scores as absent
+    }
+    __syncthreads();
+
+    // 1. scores
+    for (int r = warp; r < rows; r += kAttThreads / 32) {
+        const int i = rowi[r];
+        float dot[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) dot[g] = 0.0f;
+        if (i >= 0) {
+            const int64_t base = h * a.sh + static_cast<int64_t>(i) * a.st;
+            for (int ch = lane; ch < D; ch += 32) {
+                const float kv = kv_at<DT>(a.k, base + ch);
+#pragma unroll
+                for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g * D + ch], kv, dot[g]);
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dot[g] += __shfl_xor_sync(kFullMask, dot[g], o);
+        if (lane == 0)
+#pragma unroll
+            for (int g = 0; g < G; ++g) sc[g * kAttRows + r] = i >= 0 ? dot[g] : -INFINITY;
+    }
+    __syncthreads();
+
+    // 2. per-head chunk maximum, weights and their sum (warp g for head g)
+    if (warp < G) {
+        float* s = sc + warp * kAttRows;
+        float m = -INFINITY;
+        for (int r = lane; r < rows; r += 32) m = fmaxf(m, s[r]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+        float l = 0.0f;
+        for (int r = lane; r < rows; r += 32) {
+            const float p = m == -INFINITY ? 0.0f : expf(s[r] - m);
+            s[r] = p;
+            l += p;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(kFullMask, l, o);
+        if (lane == 0) {
+            a.pm[pbase + warp] = m;
+            a.pl[pbase + warp] = l;
+        }
+    }
+    __syncthreads();
+
+    // 3. weighted value rows
+    const int slices = kAttThreads / D;
+    const int d = tid % D, sl = tid / D;
+    if (sl < slices) {
+        float acc[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) acc[g] = 0.0f;
+        for (int r = sl; r < rows; r += slices) {
+            const int i = rowi[r];
+            if (i < 0) continue;
+            const float vv = kv_at<DT>(a.v, h * a.sh + static_cast<int64_t>(i) * a.st + d);
+#pragma unroll
+            for (int g = 0; g < G; ++g) acc[g] = fmaf(sc[g * kAttRows + r], vv, acc[g]);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) red[(sl * G + g) * D + d] = acc[g];
+    }
+    __syncthreads();
+    for (int e = tid; e < G * D; e += kAttThreads) {
+        float t = 0.0f;
+        for (int s2 = 0; s2 < slices; ++s2) t += red[s2 * G * D + e];
+        a.po[pbase * D + e] = t;
+    }
+}
+
+// Chunks -> normalised output.
+template <int G>
+__global__ void __launch_bounds__(kAttThreads)
+attend_combine_kernel(const AttArgs a)
+{
+    const int64_t h = blockIdx.x;
+    const int D = a.D;
+    for (int e = threadIdx.x; e < G * D; e += kAttThreads) {
+        const int g = e / D;
+        float m = -INFINITY;
+        for (int c = 0; c < a.chunks; ++c) m = fmaxf(m, a.pm[(h * a.chunks + c) * G + g]);
+        float l = 0.0f, o = 0.0f;
+        if (m != -INFINITY) {
+            for (int c = 0; c < a.chunks; ++c) {
+                const int64_t pc = (h * a.chunks + c) * G + g;
+                const float f = a.pm[pc] == -INFINITY ? 0.0f : expf(a.pm[pc] - m);
+                l = fmaf(a.pl[pc], f, l);
+                o = fmaf(a.po[pc * D + (e % D)], f, o);
+            }
+        }
+        a.out[h * G * D + e] = l > 0.0f ? o / l : 0.0f;
+    }
+}
+
+template <int DT, int G>
+int launch_attend_g(AttArgs a, int64_t H, cudaStream_t stream)
+{
+    const int slices = kAttThreads / a.D;
+    const size_t smem = sizeof(float) * (G * a.D + G * kAttRows + slices * G * a.D) + sizeof(int) * kAttRows;
+    cudaError_t e = cudaFuncSetAttribute(attend_chunk_kernel<DT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_status(e);
+    attend_chunk_kernel<DT, G><<<dim3(a.chunks, static_cast<unsigned>(H)), kAttThreads, smem, stream>>>(a);
+    const int st = launch_status();
+    if (st) return st;
+    attend_combine_kernel<G><<<static_cast<unsigned>(H), kAttThreads, 0, stream>>>(a);
+    return launch_status();
+}
+
+template <int DT>
+int launch_attend_dt(const AttArgs& a, int64_t H, int G, cudaStream_t stream)
+{
+    switch (G) {
+        case 1: return launch_attend_g<DT, 1>(a, H, stream);
+        case 2: return launch_attend_g<DT, 2>(a, H, stream);
+        case 3: return launch_attend_g<DT, 3>(a, H, stream);
+        case 4: return launch_attend_g<DT, 4>(a, H, stream);
+        case 5: return launch_attend_g<DT, 5>(a, H, stream);
+        case 6: return launch_attend_g<DT, 6>(a, H, stream);
+        case 7: return launch_attend_g<DT, 7>(a, H, stream);
+        default: return launch_attend_g<DT, 8>(a, H, stream);
+    }
+}
+
+int att_chunks(int64_t M) { return static_cast<int>(ceil_div(M < 1 ? 1 : M, kAttRows)); }
+
+}  // namespace
+
+size_t union_attention_workspace_bytes(int64_t H, int G, int D, int64_t M)
+{
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t cg = static_cast<size_t>(H) * att_chunks(M) * G;
+    return 2 * up(sizeof(float) * cg) + up(sizeof(float) * cg * D);
+}
+
+int launch_union_attention(const void* k, const void* v, int kv_dtype, int64_t H, int64_t n, int D, int64_t sh,
+                           int64_t st, const float* q, int G, const int32_t* uni, const int32_t* count, int64_t M,
+                           float scale, float* out, void* ws, cudaStream_t stream)
+{
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    AttArgs a{};
+    a.k = k;
+    a.v = v;
+    a.n = n;
+    a.sh = sh;
+    a.st = st;
+    a.M = M;
+    a.D = D;
+    a.q = q;
+    a.uni = uni;
+    a.count = count;
+    a.scale = scale;
+    a.chunks = att_chunks(M);
+    const size_t cg = static_cast<size_t>(H) * a.chunks * G;
+    char* base = static_cast<char*>(ws);
+    a.pm = reinterpret_cast<float*>(base);
+    a.pl = reinterpret_cast<float*>(base + up(sizeof(float) * cg));
+    a.po = reinterpret_cast<float*>(base + 2 * up(sizeof(float) * cg));
+    a.out = out;
+    if (kv_dtype == FATHOM_KEYS_BF16) return launch_attend_dt<FATHOM_KEYS_BF16>(a, H, G, stream);
+    return launch_attend_dt<FATHOM_KEYS_F32>(a, H, G, stream);
+}
+
+}  // namespace fathom

@@ -9,6 +9,7 @@ is no fallback.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -37,6 +38,7 @@ EXPORTS = (
     "fathom_pack", "fathom_plan", "fathom_plan_fixed", "fathom_scan_cand_bytes", "fathom_scan",
     "fathom_topk_workspace_bytes", "fathom_topk", "fathom_dequant_rows", "fathom_scan_topk_noalloc",
     "fathom_device_status", "fathom_calibrate_workspace_bytes", "fathom_calibrate",
+    "fathom_union_attention_workspace_bytes", "fathom_union_attention",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -82,6 +84,8 @@ def load(path: str | None = None):
         "fathom_device_status": (I, [I, P]),
         "fathom_calibrate_workspace_bytes": (SZ, [I64, I, I]),
         "fathom_calibrate": (I, [P, I, I64, I64, I, I64, I64, P, P, P, P, SZ, P]),
+        "fathom_union_attention_workspace_bytes": (SZ, [I64, I, I, I64]),
+        "fathom_union_attention": (I, [P, P, I, I64, I64, I, I64, I64, P, I, P, P, I64, ctypes.c_float, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -288,6 +292,34 @@ def calibrate(keys: torch.Tensor, n: int | None = None, with_mean: bool = True, 
     _check(lib().fathom_calibrate(_p(keys), dt, H, n, D, keys.stride(0), keys.stride(1), _p(mean), _p(sigma2),
                                   _p(cov), _p(workspace), workspace.numel(), _stream(stream)), "fathom_calibrate")
     return mean, sigma2, cov
+
+
+def union_attention_workspace_bytes(H: int, G: int, D: int, M: int) -> int:
+    return int(lib().fathom_union_attention_workspace_bytes(H, G, D, M))
+
+
+def union_attention(k_cache: torch.Tensor, v_cache: torch.Tensor, q: torch.Tensor, union_idx: torch.Tensor,
+                    union_count: torch.Tensor, scale: float | None = None, out=None, workspace=None, stream=None):
+    """Softmax attention [H][G][D] (fp32) of each query head over its group's
+    union rows of the K/V cache [H][n][D] (fp32 or bf16)."""
+    H, n, D = k_cache.shape
+    G = q.shape[1]
+    M = union_idx.shape[1]
+    if k_cache.dtype != v_cache.dtype or k_cache.shape != v_cache.shape or k_cache.stride() != v_cache.stride():
+        raise ValueError("k_cache and v_cache must share dtype, shape and strides")
+    dt = {torch.float32: KEYS_F32, torch.bfloat16: KEYS_BF16}[k_cache.dtype]
+    if k_cache.stride(2) != 1:
+        raise ValueError("the cache must be contiguous along D")
+    if out is None:
+        out = torch.empty((H, G, D), dtype=torch.float32, device=q.device)
+    need = int(lib().fathom_union_attention_workspace_bytes(H, G, D, M))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check(lib().fathom_union_attention(_p(k_cache), _p(v_cache), dt, H, n, D, k_cache.stride(0), k_cache.stride(1),
+                                        _p(q), G, _p(union_idx), _p(union_count), M, sc, _p(out), _p(workspace),
+                                        workspace.numel(), _stream(stream)), "fathom_union_attention")
+    return out
 
 
 def device_status(clear: bool = False, stream=None) -> int:

@@ -125,6 +125,17 @@ def queries(w: Workload, h0: int, h1: int, device="cpu") -> torch.Tensor:
     return torch.stack(out, 0)
 
 
+def values(w: Workload, h0: int, h1: int, device="cpu") -> torch.Tensor:
+    """Value rows of groups [h0, h1) as [h1-h0][n][D], N(0, 1), in the keys'
+    dtype: the synthetic V cache that attention over the winners reads."""
+    out = []
+    for h in range(h0, h1):
+        g = _gen(device, _group_seed(w, h, 2))
+        z = torch.randn(w.n, w.D, generator=g, device=device)
+        out.append(z.to(torch.float32 if w.kind == "gauss" else torch.bfloat16))
+    return torch.stack(out, 0)
+
+
 def calibration_sigma2(k: torch.Tensor, n_cal: int) -> torch.Tensor:
     """sigma_j^2 per group: the population variance over the first ``n_cal``
     keys of each channel, accumulated in fp64 and rounded to fp32.  This is

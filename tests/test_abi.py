@@ -60,6 +60,10 @@ def test_host_only_entry_points(lib):
     assert lib.fathom_calibrate_workspace_bytes(8, 100, 0) == 0              # unsupported D
     assert lib.fathom_calibrate_workspace_bytes(8, 128, 0) == 2 * 8 * 128 * 8
     assert lib.fathom_calibrate_workspace_bytes(8, 128, 1) == 2 * 8 * 128 * 8 + 8 * 128 * 128 * 8
+    # attention over the union: (max, weight sum) per (group, 256-row chunk, head) + the chunk outputs
+    assert lib.fathom_union_attention_workspace_bytes(288, 4, 128, 2048) == 2 * 288 * 8 * 4 * 4 + 288 * 8 * 4 * 128 * 4
+    assert lib.fathom_union_attention_workspace_bytes(1, 4, 128, 0) == 0
+    assert lib.fathom_union_attention_workspace_bytes(1, 9, 128, 64) == 0
 
 
 def test_rejections_before_any_cuda_call(lib):
@@ -84,6 +88,13 @@ def test_rejections_before_any_cuda_call(lib):
     fake = ctypes.c_void_p(256)   # never dereferenced: the size check comes first
     assert lib.fathom_calibrate(fake, 0, 2, 64, 128, 64 * 128, 128, n, fake, n, fake, 100, n) == fathom.ERR_WORKSPACE
     assert lib.fathom_calibrate(fake, 0, 2, 64, 128, 64 * 128, 128, n, n, n, fake, 1 << 20, n) == fathom.ERR_INVALID_ARG
+    ua = lib.fathom_union_attention
+    assert ua(n, n, 0, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 0, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # M = 0
+    assert ua(n, n, 2, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 8, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # dtype
+    assert ua(n, n, 0, 1, 64, 128, 64 * 128, 128, n, 9, n, n, 8, 1.0, n, n, 0, n) == fathom.ERR_UNSUPPORTED   # G = 9
+    assert ua(n, n, 0, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 8, float("nan"), n, n, 0, n) == fathom.ERR_INVALID_ARG
+    assert ua(fake, fake, 0, 2, 64, 128, 64 * 128, 128, fake, 4, fake, fake, 8, 1.0, fake, fake, 64, n) == \
+        fathom.ERR_WORKSPACE
 
 
 def test_missing_library_fails_loudly(tmp_path):

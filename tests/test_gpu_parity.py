@@ -335,3 +335,89 @@ def test_calibrate_sigma2_feeds_the_plan(fathom_gpu, orc):
     assert diff <= 2   # one-ulp fp64 summation-order cases at most
     if diff == 0:
         assert torch.equal(d_ref, d_cal) and torch.equal(a_ref, a_cal) and torch.equal(n_ref, n_cal)
+
+
+# --------------------------------------------------------------------------
+# Attention over the union of winners (byte-accounting section: the KV rows
+# of the union of the G heads' top-k are what a step fetches)
+# --------------------------------------------------------------------------
+def _attention_tolerance(k, v, q, uni, cnt):
+    """Per-element bound for the fp32 kernel against the fp64 oracle.  A
+    score is a D-term fp32 dot product (per-lane sums of D/32 terms, a
+    5-level shuffle tree, a scaled query), so |ds| <= (D/32 + 7) u S with
+    S = scale sum_j |q_j k_j| and u = 2^-24; a weight exp(s - m) then has
+    relative error <= 2 max|ds| + 4u (expf, the max, the combine), and the
+    output, a ratio of weighted sums over the c rows, adds (c + 8) u.  So
+    |out - ref| <= (4 max|ds| + 8u + (c + 8) u) sum_i p_i |v_i| / sum_i p_i."""
+    H, n, D = k.shape
+    G = q.shape[1]
+    u = 2.0 ** -24
+    tol = np.zeros((H, G, D))
+    for h in range(H):
+        c = max(0, min(int(cnt[h]), uni.shape[1]))
+        if c == 0:
+            continue
+        rows = uni[h, :c]
+        kk = k[h, rows].astype(np.float64)
+        vv = np.abs(v[h, rows].astype(np.float64))
+        s = q[h].astype(np.float64) @ kk.T / np.sqrt(D)
+        S = np.abs(q[h].astype(np.float64)) @ np.abs(kk).T / np.sqrt(D)
+        p = np.exp(s - s.max(1, keepdims=True))
+        w = (p @ vv) / p.sum(1, keepdims=True)
+        ds = (D / 32 + 7) * u * S.max(1, keepdims=True)
+        tol[h] = (4 * ds + 8 * u + (c + 8) * u) * w
+    return tol
+
+
+def _as_np(t):
+    return t.float().cpu().numpy() if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
+def test_union_attention_random_unions(fathom_gpu, orc):
+    """Ragged counts over several 256-row chunks, -1 padding, an empty and an
+    error count, and out-of-range indices (skipped) on fp32 keys."""
+    w = dataclasses.replace(inputs.TINY, name="att", H=5, n=3000, seed=15)
+    k = inputs.keys(w, 0, w.H, device=DEV)
+    v = inputs.values(w, 0, w.H, device=DEV)
+    q = inputs.queries(w, 0, w.H, device=DEV).float().contiguous()
+    M = 700
+    g = np.random.default_rng(15)
+    uni = np.full((w.H, M), -1, np.int32)
+    cnt = np.array([700, 513, 1, 0, -6], np.int32)
+    for h in range(w.H):
+        c = max(cnt[h], 0)
+        uni[h, :c] = np.sort(g.choice(w.n, c, replace=False))
+    bad = uni.copy()
+    bad[1, 5] = w.n + 3          # outside the cache: skipped by the kernel
+    out = fathom_gpu.union_attention(k, v, q, torch.from_numpy(bad).to(DEV), torch.from_numpy(cnt).to(DEV))
+    torch.cuda.synchronize()
+    ref_uni = uni.copy()
+    ref_cnt = cnt.copy()
+    ref_uni[1, 5:512] = ref_uni[1, 6:513]   # the same rows without the skipped entry
+    ref_uni[1, 512] = -1
+    ref_cnt[1] = 512
+    ref = orc.union_attention(_as_np(k), _as_np(v), _as_np(q), ref_uni, ref_cnt)
+    got = out.cpu().numpy().astype(np.float64)
+    tol = _attention_tolerance(_as_np(k), _as_np(v), _as_np(q), ref_uni, ref_cnt)
+    assert np.all(np.abs(got - ref) <= tol + 1e-30), np.max(np.abs(got - ref) - tol)
+    assert not np.any(got[3]) and not np.any(got[4])
+
+
+def test_union_attention_after_a_step(fathom_gpu, orc):
+    """The union a 48-bit candidate step selects on a Qwen3-8B-shaped layer
+    (bf16 K/V, up to 2048 rows per group), attended over and checked against
+    the oracle on the same rows."""
+    w = dataclasses.replace(inputs.LAYER_32K, H=3, seed=16)
+    k, q, s2 = make(w)
+    v = inputs.values(w, 0, w.H, device=DEV)
+    planes, scales = fathom_gpu.pack(k)
+    step = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, budget=48)
+    _, uni, cnt = step.run(q)
+    out = fathom_gpu.union_attention(k, v, q, uni, cnt)
+    torch.cuda.synchronize()
+    un, cn = uni.cpu().numpy(), cnt.cpu().numpy()
+    assert np.all(cn > w.k)
+    ref = orc.union_attention(keys_for_oracle(k), keys_for_oracle(v), _as_np(q), un, cn)
+    tol = _attention_tolerance(_as_np(k), _as_np(v), _as_np(q), un, cn)
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= tol + 1e-30), np.max(np.abs(got - ref) - tol)
