@@ -52,6 +52,8 @@ def _lib():
         lib.orc_dequant_rows.argtypes = [P, P, I64, I, I64, I64, P, I64, P, I, P]
         lib.orc_calibrate.restype = I
         lib.orc_calibrate.argtypes = [P, I, I64, I64, I, I64, I64, P, P, P]
+        lib.orc_pack_nibbles.restype = I
+        lib.orc_pack_nibbles.argtypes = [P, I, I64, I64, I, I64, I64, P, I64]
         lib.orc_union_attention.restype = I
         lib.orc_union_attention.argtypes = [P, P, I, I64, I64, I, I64, I64, P, I, P, P, I64, ctypes.c_double, P]
         _LIB = lib
@@ -231,3 +233,16 @@ def union_attention(k: np.ndarray, v: np.ndarray, q: np.ndarray, uni: np.ndarray
     _check(_lib().orc_union_attention(_ptr(k), _ptr(v), dt, H, n, D, n * D, D, _ptr(q), G, _ptr(uni), _ptr(count),
                                       M, sc, _ptr(out)), "union_attention")
     return out
+
+
+def pack_nibbles(keys: np.ndarray, nb_stride: int | None = None) -> np.ndarray:
+    """The 4-bit codes of ``pack`` stored whole: uint64 [H][D][4][nb_stride],
+    word w of a block holding its tokens 16w..16w+15, 4 bits each."""
+    keys = np.ascontiguousarray(keys)
+    dt = {np.dtype(np.float32): 0, np.dtype(np.uint16): 1}[keys.dtype]
+    H, n, D = keys.shape
+    nb = (n + 63) // 64
+    nbs = nb if nb_stride is None else int(nb_stride)
+    nib = np.zeros((H, D, 4, nbs), dtype=np.uint64)
+    _check(_lib().orc_pack_nibbles(_ptr(keys), dt, H, n, D, n * D, D, _ptr(nib), nbs), "pack_nibbles")
+    return nib

@@ -36,6 +36,9 @@
  *   orc_union_attention  softmax attention of each query head over its KV
  *                      head's union of winner rows (byte-accounting
  *                      section: the winner rows a step fetches)
+ *   orc_pack_nibbles   the same 4-bit codes stored whole, 4 bits per token
+ *                      (the fixed-depth scans' 4-bit coordinates of the
+ *                      byte-accounting section), 16 tokens per 64-bit word
  */
 #include <math.h>
 #include <stdint.h>
@@ -522,5 +525,46 @@ int orc_union_attention(const void* kc, const void* vc, int kv_dtype, int64_t H,
         }
     }
     free(sc);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Nibble store of the same codes (byte-accounting section: a fixed-depth */
+/* scan reads each chosen coordinate's whole 4-bit code).  Word w of     */
+/* block b of channel j holds tokens 64b + 16w .. 64b + 16w + 15, token  */
+/* 64b + 16w + e in bits 4e .. 4e + 3.  Layout [H][D][4][nb_stride] like  */
+/* the planes: row (h, j, w) is contiguous along the blocks.  Padding    */
+/* tokens (past n) hold code 0.  Scales are those of orc_pack.           */
+/* ------------------------------------------------------------------ */
+int orc_pack_nibbles(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
+                     int64_t stride_h, int64_t stride_tok, uint64_t* nib, int64_t nb_stride)
+{
+    if (!keys || !nib || H < 0 || n < 0 || D <= 0) return ORC_EINVAL;
+    int64_t nb = (n + 63) / 64;
+    if (nb_stride < nb) return ORC_EINVAL;
+    for (int64_t h = 0; h < H; ++h) {
+        for (int j = 0; j < D; ++j) {
+            for (int64_t b = 0; b < nb; ++b) {
+                double kv[64];
+                int cnt = 0;
+                double m = 0.0;
+                for (int i = 0; i < 64; ++i) {
+                    int64_t tok = b * 64 + i;
+                    if (tok >= n) break;
+                    int64_t off = h * stride_h + tok * stride_tok + j;
+                    double v = key_dtype == 1 ? orc_bf16_value(((const uint16_t*)keys)[off])
+                                              : (double)((const float*)keys)[off];
+                    kv[i] = v;
+                    if (fabs(v) > m) m = fabs(v);
+                    cnt++;
+                }
+                double s = orc_fp16_value(orc_fp16_bits(m));
+                uint64_t w[4] = {0, 0, 0, 0};
+                for (int i = 0; i < cnt; ++i)
+                    w[i / 16] |= (uint64_t)orc_code4(kv[i], s) << (4 * (i % 16));
+                for (int p = 0; p < 4; ++p) nib[(((h * D) + j) * 4 + p) * nb_stride + b] = w[p];
+            }
+        }
+    }
     return ORC_OK;
 }

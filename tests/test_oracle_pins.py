@@ -577,3 +577,39 @@ def test_union_attention_special_cases(orc):
     assert np.array_equal(orc.union_attention(kb, vb, q, rows, np.full(H, 40, np.int32)),
                           orc.union_attention(np.ascontiguousarray(kf), np.ascontiguousarray(vf), q, rows,
                                               np.full(H, 40, np.int32)))
+
+
+# --------------------------------------------------------------------------
+# Nibble store (byte-accounting section: the fixed-depth scans' whole 4-bit
+# coordinates)
+# --------------------------------------------------------------------------
+def test_nibbles_hold_the_plane_codes(orc):
+    """Token i's nibble is the 4-bit code whose bits the four planes hold
+    (plane p = bit 3 - p), for every token, with zero past n; and with all
+    four planes read the scan equals the nibble code's mid-rise value times
+    the query (decoded here straight from the nibbles)."""
+    rng = np.random.default_rng(21)
+    H, n, D = 2, 300, 8
+    k = (rng.standard_normal((H, n, D)) * np.exp(rng.normal(0, 1, D))).astype(np.float32)
+    planes, scales = orc.pack(k)
+    nib = orc.pack_nibbles(k)
+    nb = (n + 63) // 64
+    for h in range(H):
+        for j in range(D):
+            for b in range(nb):
+                for i in range(64):
+                    code_p = sum(((int(planes[h, j, p, b]) >> i) & 1) << (3 - p) for p in range(4))
+                    code_n = (int(nib[h, j, i // 16, b]) >> (4 * (i % 16))) & 15
+                    assert code_n == code_p
+                    if b * 64 + i >= n:
+                        assert code_n == 0
+    q = rng.standard_normal((H, 4, D)).astype(np.float32)
+    depth = np.full((H, D), 4, np.uint8)
+    sc = orc.scan(planes, scales, depth, q, n, with_l1=False)
+    s = np.array([[orc.fp16_value(int(x)) for x in row] for row in scales.reshape(H * D, nb)]).reshape(H, D, nb)
+    for h in range(H):
+        for i in range(n):
+            b = i // 64
+            codes = np.array([(int(nib[h, j, (i % 64) // 16, b]) >> (4 * (i % 16))) & 15 for j in range(D)])
+            khat = (codes - 7.5) * s[h, :, b] / 8.0
+            assert np.allclose(sc[h, :, i], q[h].astype(np.float64) @ khat, rtol=1e-12, atol=1e-12)
