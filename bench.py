@@ -542,6 +542,30 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     nrows = int(cnt.clamp(min=0).sum().item())
     out["reconstruct_union_rows"] = {"ms": tot / 5, "rows": nrows, "rows_per_s": nrows / (tot / 5 / 1e3),
                                      "out_GBps": nrows * w.D * 4 / (tot / 5 / 1e3) / 1e9}
+    # The fixed 136-bit scan over the nibble store (whole 4-bit codes): the
+    # same bytes as the plane scan at depth 4, decoded from nibbles.
+    nib = fathom.nibbles_from_planes(planes, w.n)
+    stn = fathom.Step(planes, scales, w.n, sigma2, w.G, k, fixed_r=32, nibbles=nib)
+
+    def onen(ev, st=stn):
+        st.run_plan(q)
+        st.run_prepare(q)
+        if ev is not None:
+            ev[0].record()
+        st.run_filter(q)
+        if ev is not None:
+            ev[1].record()
+        st.run_topk()
+    onen(None)
+    torch.cuda.synchronize(device)
+    fbn = stn.repair(q)
+    alg, bits, na = plan_bytes(stn, w)
+    tot, fk = time_steps(onen, 5, 2, device, kernel_events=True)
+    fm = statistics.fmean(fk)
+    out["nibble136_r32"] = {"ms_per_step": tot / 5, "scan_ms": fm, "scan_GBps": alg / (fm / 1e3) / 1e9,
+                            "read_bits_per_token": alg * 8 / (w.H * w.n), "fallback_groups": fbn}
+    del stn, nib
+    torch.cuda.empty_cache()
     # Attention of the step's query heads over their union rows, for the
     # first layer's 8 groups (their full-precision K/V cache regenerated).
     from long_context_decode_bit_b200 import inputs as _inp

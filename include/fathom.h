@@ -264,6 +264,35 @@ int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
                 fathom_stream_t stream);
 
 /*
+ * fathom_nibbles_from_planes -- the same 4-bit codes stored whole: for each
+ * (group, channel, block) four 64-bit words, word w holding tokens
+ * 16w .. 16w+15 of the block, token 16w + e in bits 4e .. 4e+3.  Layout
+ * [H][D][4][nb_stride], like the planes (a row (h, j, w) is contiguous along
+ * the blocks), and the scales are the planes' own.  This is the store a
+ * fixed-depth scan reads (先算一笔字节账: 32 coordinates at 4 bits plus a
+ * block scale), kept as a comparator: its bytes per read coordinate equal
+ * the planes' at depth 4, so the two scans differ only in decoding.
+ *
+ *   planes      DEVICE, as written by fathom_pack.
+ *   nibbles     DEVICE out, uint64 [H][D][4][nb_stride].
+ */
+int fathom_nibbles_from_planes(const uint64_t* planes, int64_t H, int D, int64_t n, int64_t nb_stride,
+                               uint64_t* nibbles, fathom_stream_t stream);
+
+/*
+ * fathom_scan_nibbles -- fathom_scan over the nibble store: every active
+ * channel is read whole (4 bits; the plan's depths are ignored), so it
+ * computes the scores of fathom_scan with every active depth at 4, bit for
+ * bit.  Arguments, modes, outputs and errors are fathom_scan's, with
+ * `nibbles` in place of `planes`.
+ */
+int fathom_scan_nibbles(const uint64_t* nibbles, const uint16_t* scales, int64_t H, int D,
+                        int64_t n, int64_t nb_stride, const uint16_t* active,
+                        const int32_t* n_active, const float* q, int G, int mode,
+                        float* scores, void* cand, size_t cand_bytes, int k,
+                        fathom_stream_t stream);
+
+/*
  * fathom_topk_workspace_bytes -- scratch fathom_topk needs (HOST call).
  */
 size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k);

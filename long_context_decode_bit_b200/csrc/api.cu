@@ -14,7 +14,7 @@ int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits, 
                       int32_t* n_active, cudaStream_t stream);
 int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
                 const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
-                void* cand, int k, cudaStream_t stream);
+                void* cand, int k, bool nib, cudaStream_t stream);
 int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
                 int32_t* union_idx, int32_t* union_count, cudaStream_t stream);
 
@@ -67,6 +67,70 @@ int check_device_ptr(const void* p)
 }
 
 bool dims_ok(int D, int G) { return D >= 32 && D <= kMaxD && D % 32 == 0 && G >= 1 && G <= kMaxG; }
+
+#define FATHOM_TRY_IN(expr)              \
+    do {                                 \
+        const int _st = (expr);          \
+        if (_st != FATHOM_OK) return _st; \
+    } while (0)
+
+int scan_entry(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
+               const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
+               void* cand, size_t cand_bytes, int k, bool nib, fathom_stream_t stream)
+{
+    if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
+    if (mode < FATHOM_SCAN_DENSE || mode > FATHOM_SCAN_FILTER) return FATHOM_ERR_INVALID_ARG;
+    if (H == 0 || n == 0) return FATHOM_OK;
+    const int64_t nb = ceil_div(n, kBlockTokens);
+    if (nb_stride < nb) return FATHOM_ERR_INVALID_ARG;
+    if ((nb_stride & 7) || !aligned(planes, 16) || !aligned(scales, 16) || !aligned(active, 2) ||
+        !aligned(n_active, 4) || !aligned(q, 4))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY_IN(check_device_ptr(planes));
+    FATHOM_TRY_IN(check_device_ptr(scales));
+    FATHOM_TRY_IN(check_device_ptr(active));
+    FATHOM_TRY_IN(check_device_ptr(n_active));
+    FATHOM_TRY_IN(check_device_ptr(q));
+    if (mode == FATHOM_SCAN_DENSE) {
+        if (!aligned(scores, 4)) return FATHOM_ERR_UNSUPPORTED;
+        FATHOM_TRY_IN(check_device_ptr(scores));
+    } else {
+        if (k < 1 || k > n) return FATHOM_ERR_INVALID_ARG;
+        if (k > kMaxCandK) return FATHOM_ERR_UNSUPPORTED;
+        if (!aligned(cand, 16)) return FATHOM_ERR_UNSUPPORTED;
+        FATHOM_TRY_IN(check_device_ptr(cand));
+        if (cand_bytes < cand_layout(H, G, n, k).total) return FATHOM_ERR_WORKSPACE;
+    }
+    return launch_scan(planes, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, k, nib,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+// One thread per (group, channel, block): the four plane words -> the four
+// nibble words of the same codes.
+__global__ void nibbles_kernel(const uint64_t* __restrict__ planes, int64_t rows, int64_t nb, int64_t nb_stride,
+                               uint64_t* __restrict__ nib)
+{
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= rows * nb) return;
+    const int64_t r = t / nb, b = t % nb;   // r = h * D + j
+    uint64_t p[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) p[q] = planes[(r * 4 + q) * nb_stride + b];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        uint64_t out = 0;
+        for (int e = 0; e < 16; ++e) {
+            const int i = 16 * w + e;
+            uint64_t c = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) c |= ((p[q] >> i) & 1ull) << (3 - q);
+            out |= c << (4 * e);
+        }
+        nib[(r * 4 + w) * nb_stride + b] = out;
+    }
+}
+
 
 }  // namespace
 }  // namespace fathom
@@ -237,32 +301,33 @@ int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
                 const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
                 void* cand, size_t cand_bytes, int k, fathom_stream_t stream)
 {
-    if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
-    if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
-    if (mode < FATHOM_SCAN_DENSE || mode > FATHOM_SCAN_FILTER) return FATHOM_ERR_INVALID_ARG;
+    return fathom::scan_entry(planes, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, cand_bytes, k,
+                      false, stream);
+}
+
+int fathom_scan_nibbles(const uint64_t* nibbles, const uint16_t* scales, int64_t H, int D, int64_t n,
+                        int64_t nb_stride, const uint16_t* active, const int32_t* n_active, const float* q, int G,
+                        int mode, float* scores, void* cand, size_t cand_bytes, int k, fathom_stream_t stream)
+{
+    return fathom::scan_entry(nibbles, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, cand_bytes, k,
+                      true, stream);
+}
+
+int fathom_nibbles_from_planes(const uint64_t* planes, int64_t H, int D, int64_t n, int64_t nb_stride,
+                               uint64_t* nibbles, fathom_stream_t stream)
+{
+    if (H < 0 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
     if (H == 0 || n == 0) return FATHOM_OK;
     const int64_t nb = ceil_div(n, kBlockTokens);
     if (nb_stride < nb) return FATHOM_ERR_INVALID_ARG;
-    if ((nb_stride & 7) || !aligned(planes, 16) || !aligned(scales, 16) || !aligned(active, 2) ||
-        !aligned(n_active, 4) || !aligned(q, 4))
-        return FATHOM_ERR_UNSUPPORTED;
+    if (!aligned(planes, 8) || !aligned(nibbles, 8)) return FATHOM_ERR_UNSUPPORTED;
     FATHOM_TRY(check_device_ptr(planes));
-    FATHOM_TRY(check_device_ptr(scales));
-    FATHOM_TRY(check_device_ptr(active));
-    FATHOM_TRY(check_device_ptr(n_active));
-    FATHOM_TRY(check_device_ptr(q));
-    if (mode == FATHOM_SCAN_DENSE) {
-        if (!aligned(scores, 4)) return FATHOM_ERR_UNSUPPORTED;
-        FATHOM_TRY(check_device_ptr(scores));
-    } else {
-        if (k < 1 || k > n) return FATHOM_ERR_INVALID_ARG;
-        if (k > kMaxCandK) return FATHOM_ERR_UNSUPPORTED;
-        if (!aligned(cand, 16)) return FATHOM_ERR_UNSUPPORTED;
-        FATHOM_TRY(check_device_ptr(cand));
-        if (cand_bytes < cand_layout(H, G, n, k).total) return FATHOM_ERR_WORKSPACE;
-    }
-    return launch_scan(planes, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, k,
-                       reinterpret_cast<cudaStream_t>(stream));
+    FATHOM_TRY(check_device_ptr(nibbles));
+    const int64_t total = H * D * nb;
+    fathom::nibbles_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        planes, H * D, nb, nb_stride, nibbles);
+    return launch_status();
 }
 
 size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k)

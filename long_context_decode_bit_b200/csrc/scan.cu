@@ -86,6 +86,7 @@ struct ScanArgs {
     int tiles_per_cta;
     int mode;
     int32_t* fault;            // device fault word: set when a ring wait ran out
+    bool nib;                  // `planes` is the nibble store, read at 4 bits
 };
 
 // Heads are handled in pairs for the packed FMA; odd G gets a zero pad.
@@ -217,10 +218,24 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr)
 }
 
 // One channel of depth T for the lane's block: 8 tokens x G heads.
-// wrow: shared address of the channel's first plane row at the lane's block
-// column; cf: shared address of its head-pair coefficients for that block.
-// The 8 token values of one channel of depth T for the lane's block.
-template <int T>
+// The whole 4-bit code c in nibble l of `x` as the exact odd integer
+// 2c - 15: one rotation moves the nibble to mantissa bits 19..22 of 1.0f,
+// giving 1 + c/16, and one FMA with exact constants finishes (32 + 2c - 47).
+// Token values of the nibble store (see channel_values).
+__device__ __forceinline__ float value_nibble(uint32_t x, int l)
+{
+    const uint32_t r = __funnelshift_l(x, x, (19 - 4 * l) & 31);
+    const float f = __uint_as_float((r & 0x00780000u) | 0x3F800000u);   // 1 + c/16
+    return __fmaf_rn(f, 32.0f, -47.0f);
+}
+
+// The 8 token values of one channel of depth T for the lane's block.  wrow:
+// shared address of the channel's first row at the lane's block column.
+// With NIB the rows are the nibble store's four words per block (word w:
+// tokens 16w..16w+15, 4 bits each) and T is 4: slot s of the lane (token
+// l + 8s, or 32 + l + 8(s - 4)) is nibble l of the 32-bit half s & 1 of
+// word s >> 1.
+template <int T, bool NIB>
 __device__ __forceinline__ void channel_values(uint32_t wrow, int l, float (&v)[8])
 {
     uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
@@ -230,7 +245,13 @@ __device__ __forceinline__ void channel_values(uint32_t wrow, int l, float (&v)[
         lo[p] = x.x;
         hi[p] = x.y;
     }
-    if (T == 1) {
+    if (NIB) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            v[2 * w] = value_nibble(lo[w], l);
+            v[2 * w + 1] = value_nibble(hi[w], l);
+        }
+    } else if (T == 1) {
         values_depth1(lo[0], l, *reinterpret_cast<float(*)[4]>(&v[0]));
         values_depth1(hi[0], l, *reinterpret_cast<float(*)[4]>(&v[4]));
     } else {
@@ -239,7 +260,8 @@ __device__ __forceinline__ void channel_values(uint32_t wrow, int l, float (&v)[
     }
 }
 
-// acc += coefficient * value for the 8 tokens x G heads of one channel.
+// acc += coefficient * value for the 8 tokens x G heads of one channel.  cf:
+// shared address of the channel's head-pair coefficients for the block.
 template <int G>
 __device__ __forceinline__ void channel_macs(const float (&v)[8], uint32_t cf, float2 (&acc)[8][head_pairs<G>()])
 {
@@ -261,14 +283,14 @@ __device__ __forceinline__ void channel_macs(const float (&v)[8], uint32_t cf, f
 }
 
 // All channels of depth T in a chunk.
-template <int G, int T>
+template <int G, int T, bool NIB>
 __device__ __forceinline__ void depth_class(uint32_t& wrow, uint32_t& cf, int count, int l,
                                             float2 (&acc)[8][head_pairs<G>()])
 {
     constexpr uint32_t kCf = kBlocksPerWarp * coef_pairs<G>() * 8;
     for (int i = 0; i < count; ++i) {
         float v[8];
-        channel_values<T>(wrow, l, v);
+        channel_values<T, NIB>(wrow, l, v);
         channel_macs<G>(v, cf, acc);
         wrow += T * kRowBytes;
         cf += kCf;
@@ -285,7 +307,7 @@ __device__ __forceinline__ float acc_at(const float2 (&acc)[8][head_pairs<G>()],
 #define FATHOM_SCAN_MIN_CTAS (kScanTileBlocks == 16 ? 3 : 2)
 #endif
 
-template <int G>
+template <int G, bool NIB>
 __global__ void __launch_bounds__(kScanThreads, FATHOM_SCAN_MIN_CTAS)
 scan_kernel(const ScanArgs a)
 {
@@ -303,7 +325,7 @@ scan_kernel(const ScanArgs a)
     for (int i = tid; i < na; i += kScanThreads) {
         const uint16_t e = a.active[h * D + i];
         const int j = e & 0xFF;
-        int tt = min(e >> 8, kPlanes);
+        int tt = NIB ? kPlanes : min(e >> 8, kPlanes);   // the nibble store is read whole
         if (j >= D) tt = 0;       // malformed entry: read nothing
         S.rowsrc[i] = static_cast<uint16_t>(j | (tt << 8));   // staging area until the sort is done
     }
@@ -471,10 +493,10 @@ scan_kernel(const ScanArgs a)
                       n1 = S.chunk_cnt[ck][3];
             uint32_t wrow = static_cast<uint32_t>(__cvta_generic_to_shared(&S.words[st][blk]));  // row 0, lane's block
             uint32_t cf = static_cast<uint32_t>(__cvta_generic_to_shared(wcoef + bl * coef_pairs<G>()));
-            depth_class<G, 4>(wrow, cf, n4, l, acc);
-            depth_class<G, 3>(wrow, cf, n3, l, acc);
-            depth_class<G, 2>(wrow, cf, n2, l, acc);
-            depth_class<G, 1>(wrow, cf, n1, l, acc);
+            depth_class<G, 4, NIB>(wrow, cf, n4, l, acc);
+            depth_class<G, 3, NIB>(wrow, cf, n3, l, acc);
+            depth_class<G, 2, NIB>(wrow, cf, n2, l, acc);
+            depth_class<G, 1, NIB>(wrow, cf, n1, l, acc);
         }
         __syncwarp();   // the warp's coefficient table may be rebuilt after this
 
@@ -554,11 +576,11 @@ scan_kernel(const ScanArgs a)
     }
 }
 
-template <int G>
+template <int G, bool NIB>
 int launch_scan_g(ScanArgs a, int64_t ltiles, unsigned H, cudaStream_t stream)
 {
     const size_t smem = sizeof(SharedScan<G>);
-    const cudaError_t e = cudaFuncSetAttribute(scan_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(scan_kernel<G, NIB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_status(e);
     // Several tiles per CTA amortise the per-CTA plan set-up: as many as
@@ -572,22 +594,28 @@ int launch_scan_g(ScanArgs a, int64_t ltiles, unsigned H, cudaStream_t stream)
     const int64_t per = ceil_div(ltiles * static_cast<int64_t>(H), slots);
     a.tiles_per_cta = static_cast<int>(per < 1 ? 1 : (per > FATHOM_SCAN_TILES_CAP ? FATHOM_SCAN_TILES_CAP : per));
     const unsigned gx = static_cast<unsigned>(ceil_div(ltiles, a.tiles_per_cta));
-    scan_kernel<G><<<dim3(gx, H), kScanThreads, smem, stream>>>(a);
+    scan_kernel<G, NIB><<<dim3(gx, H), kScanThreads, smem, stream>>>(a);
     return launch_status();
+}
+
+template <bool NIB>
+int launch_scan_layout(const ScanArgs& a, int G, int64_t ltiles, unsigned H, cudaStream_t stream)
+{
+    switch (G) {
+        case 1: return launch_scan_g<1, NIB>(a, ltiles, H, stream);
+        case 2: return launch_scan_g<2, NIB>(a, ltiles, H, stream);
+        case 3: return launch_scan_g<3, NIB>(a, ltiles, H, stream);
+        case 4: return launch_scan_g<4, NIB>(a, ltiles, H, stream);
+        case 5: return launch_scan_g<5, NIB>(a, ltiles, H, stream);
+        case 6: return launch_scan_g<6, NIB>(a, ltiles, H, stream);
+        case 7: return launch_scan_g<7, NIB>(a, ltiles, H, stream);
+        default: return launch_scan_g<8, NIB>(a, ltiles, H, stream);
+    }
 }
 
 int launch_scan_mode(const ScanArgs& a, int G, int64_t ltiles, unsigned H, cudaStream_t stream)
 {
-    switch (G) {
-        case 1: return launch_scan_g<1>(a, ltiles, H, stream);
-        case 2: return launch_scan_g<2>(a, ltiles, H, stream);
-        case 3: return launch_scan_g<3>(a, ltiles, H, stream);
-        case 4: return launch_scan_g<4>(a, ltiles, H, stream);
-        case 5: return launch_scan_g<5>(a, ltiles, H, stream);
-        case 6: return launch_scan_g<6>(a, ltiles, H, stream);
-        case 7: return launch_scan_g<7>(a, ltiles, H, stream);
-        default: return launch_scan_g<8>(a, ltiles, H, stream);
-    }
+    return a.nib ? launch_scan_layout<true>(a, G, ltiles, H, stream) : launch_scan_layout<false>(a, G, ltiles, H, stream);
 }
 
 }  // namespace
@@ -637,9 +665,10 @@ CandLayout cand_layout(int64_t H, int G, int64_t n, int k)
 
 int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n,
                 int64_t nb_stride, const uint16_t* active, const int32_t* n_active, const float* q,
-                int G, int mode, float* scores, void* cand, int k, cudaStream_t stream)
+                int G, int mode, float* scores, void* cand, int k, bool nib, cudaStream_t stream)
 {
     ScanArgs a{};
+    a.nib = nib;
     {
         const int st = device_fault_word(&a.fault);
         if (st) return st;

@@ -39,6 +39,7 @@ EXPORTS = (
     "fathom_topk_workspace_bytes", "fathom_topk", "fathom_dequant_rows", "fathom_scan_topk_noalloc",
     "fathom_device_status", "fathom_calibrate_workspace_bytes", "fathom_calibrate",
     "fathom_union_attention_workspace_bytes", "fathom_union_attention",
+    "fathom_nibbles_from_planes", "fathom_scan_nibbles",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -85,6 +86,8 @@ def load(path: str | None = None):
         "fathom_calibrate_workspace_bytes": (SZ, [I64, I, I]),
         "fathom_calibrate": (I, [P, I, I64, I64, I, I64, I64, P, P, P, P, SZ, P]),
         "fathom_union_attention_workspace_bytes": (SZ, [I64, I, I, I64]),
+        "fathom_nibbles_from_planes": (I, [P, I64, I, I64, I64, P, P]),
+        "fathom_scan_nibbles": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, SZ, I, P]),
         "fathom_union_attention": (I, [P, P, I, I64, I64, I, I64, I64, P, I, P, P, I64, ctypes.c_float, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
@@ -196,23 +199,35 @@ def plan_fixed(q: torch.Tensor, r: int, out=None, stream=None, bits: int = 4):
 
 
 def scan(planes, scales, n: int, active, n_active, q, mode: int = SCAN_DENSE, k: int = 0,
-         scores=None, cand=None, stream=None):
-    """Scores [H][G][n] (DENSE) or the candidate buffer (CANDIDATE)."""
+         scores=None, cand=None, stream=None, nibbles: bool = False):
+    """Scores [H][G][n] (DENSE) or the candidate buffer (CANDIDATE).  With
+    ``nibbles`` the first argument is the nibble store (every active channel
+    read at 4 bits)."""
     H, G, D = q.shape
     nbs = planes.shape[-1]
+    fn, name = (lib().fathom_scan_nibbles, "fathom_scan_nibbles") if nibbles else (lib().fathom_scan, "fathom_scan")
     if mode == SCAN_DENSE:
         if scores is None:
             scores = torch.empty((H, G, n), dtype=torch.float32, device=q.device)
-        _check(lib().fathom_scan(_p(planes), _p(scales), H, D, n, nbs, _p(active), _p(n_active), _p(q), G,
-                                 SCAN_DENSE, _p(scores), None, 0, int(k), _stream(stream)), "fathom_scan")
+        _check(fn(_p(planes), _p(scales), H, D, n, nbs, _p(active), _p(n_active), _p(q), G,
+                  SCAN_DENSE, _p(scores), None, 0, int(k), _stream(stream)), name)
         return scores
     nbytes = scan_cand_bytes(H, G, n, k)
     if cand is None:
         cand = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    _check(lib().fathom_scan(_p(planes), _p(scales), H, D, n, nbs, _p(active), _p(n_active), _p(q), G,
-                             int(mode), None, _p(cand), cand.numel() * cand.element_size(), int(k),
-                             _stream(stream)), "fathom_scan")
+    _check(fn(_p(planes), _p(scales), H, D, n, nbs, _p(active), _p(n_active), _p(q), G,
+              int(mode), None, _p(cand), cand.numel() * cand.element_size(), int(k), _stream(stream)), name)
     return cand
+
+
+def nibbles_from_planes(planes, n: int, out=None, stream=None):
+    """The nibble store [H][D][4][nb_stride] of the codes the planes hold."""
+    H, D, _, nbs = planes.shape
+    if out is None:
+        out = torch.empty_like(planes)
+    _check(lib().fathom_nibbles_from_planes(_p(planes), H, D, n, nbs, _p(out), _stream(stream)),
+           "fathom_nibbles_from_planes")
+    return out
 
 
 def topk(H: int, G: int, n: int, k: int, scores=None, cand=None, out=None, workspace=None, stream=None):
@@ -336,11 +351,15 @@ class Step:
     """One decode step of the scan over a resident index: plan -> candidate
     scan -> top-k + union, with the dense rerun for any group whose
     candidate pass could not prove its top-k exact.  Buffers are allocated
-    once; ``run`` launches only library kernels."""
+    once; ``run`` launches only library kernels.  With ``nibbles`` the scans
+    read that nibble store (every active channel whole) instead of the
+    planes."""
 
     def __init__(self, planes, scales, n: int, sigma2, G: int, k: int, budget=48, fixed_r: int | None = None,
-                 fixed_bits: int = 4):
+                 fixed_bits: int = 4, nibbles=None):
         self.planes, self.scales, self.n, self.sigma2, self.k = planes, scales, n, sigma2, k
+        self.nibbles = nibbles
+        self.store = planes if nibbles is None else nibbles
         self.H, self.D = sigma2.shape
         self.G = G
         self.budget = budget
@@ -367,11 +386,13 @@ class Step:
 
     def run_prepare(self, q):
         _, active, n_active, _ = self.plan_out
-        return scan(self.planes, self.scales, self.n, active, n_active, q, SCAN_PREPARE, self.k, cand=self.cand)
+        return scan(self.store, self.scales, self.n, active, n_active, q, SCAN_PREPARE, self.k, cand=self.cand,
+                    nibbles=self.nibbles is not None)
 
     def run_filter(self, q):
         _, active, n_active, _ = self.plan_out
-        return scan(self.planes, self.scales, self.n, active, n_active, q, SCAN_FILTER, self.k, cand=self.cand)
+        return scan(self.store, self.scales, self.n, active, n_active, q, SCAN_FILTER, self.k, cand=self.cand,
+                    nibbles=self.nibbles is not None)
 
     def run_scan(self, q):
         self.run_prepare(q)
@@ -399,6 +420,7 @@ class Step:
         _, active, n_active, _ = self.plan_out
         for h in bad:
             sl = slice(h, h + 1)
-            sc = scan(self.planes[sl], self.scales[sl], self.n, active[sl], n_active[sl], q[sl], SCAN_DENSE)
+            sc = scan(self.store[sl], self.scales[sl], self.n, active[sl], n_active[sl], q[sl], SCAN_DENSE,
+                      nibbles=self.nibbles is not None)
             topk(1, self.G, self.n, self.k, scores=sc, out=(idx[sl], uni[sl], cnt[sl]))
         return len(bad)

@@ -88,6 +88,10 @@ def test_rejections_before_any_cuda_call(lib):
     fake = ctypes.c_void_p(256)   # never dereferenced: the size check comes first
     assert lib.fathom_calibrate(fake, 0, 2, 64, 128, 64 * 128, 128, n, fake, n, fake, 100, n) == fathom.ERR_WORKSPACE
     assert lib.fathom_calibrate(fake, 0, 2, 64, 128, 64 * 128, 128, n, n, n, fake, 1 << 20, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_scan_nibbles(n, n, 1, 128, 100, 2, n, n, n, 4, 5, n, n, 0, 1, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_scan_nibbles(n, n, 1, 100, 100, 2, n, n, n, 4, 0, n, n, 0, 1, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_nibbles_from_planes(n, 1, 48, 100, 2, n, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_nibbles_from_planes(n, 1, 128, 1000, 15, n, n) == fathom.ERR_INVALID_ARG   # stride < nb
     ua = lib.fathom_union_attention
     assert ua(n, n, 0, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 0, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # M = 0
     assert ua(n, n, 2, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 8, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # dtype

@@ -421,3 +421,36 @@ def test_union_attention_after_a_step(fathom_gpu, orc):
     tol = _attention_tolerance(_as_np(k), _as_np(v), _as_np(q), un, cn)
     got = out.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - ref) <= tol + 1e-30), np.max(np.abs(got - ref) - tol)
+
+
+# --------------------------------------------------------------------------
+# Nibble store comparator (byte-accounting section: the fixed-depth scans
+# read 32 coordinates' whole 4-bit codes)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [inputs.TINY, dataclasses.replace(inputs.LAYER_32K, name="nib-ragged", H=3, n=9001,
+                                                                seed=17)], ids=["tiny", "qk-ragged"])
+def test_nibbles_bit_exact_and_scan_equals_full_depth(fathom_gpu, orc, w):
+    """The nibble store built from the GPU planes equals the oracle's nibble
+    pack of the keys; its dense scan equals the plane scan at full depth
+    bit for bit (same coefficients, same odd integers, same FMA order) and
+    the oracle within tolerance; its candidate step picks the same top-k."""
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    nib = fathom_gpu.nibbles_from_planes(planes, w.n)
+    torch.cuda.synchronize()
+    ref = orc.pack_nibbles(keys_for_oracle(k), nb_stride=planes.shape[-1])
+    nb = w.nb
+    assert np.array_equal(np_u64(nib)[..., :nb], ref[..., :nb])
+    depth, active, na = fathom_gpu.plan_fixed(q, 32)
+    s_nib = fathom_gpu.scan(nib, scales, w.n, active, na, q, nibbles=True)
+    s_pl = fathom_gpu.scan(planes, scales, w.n, active, na, q)
+    torch.cuda.synchronize()
+    assert torch.equal(s_nib, s_pl)
+    o_scores, o_l1 = orc.scan(np_u64(planes), np_u16(scales), depth.cpu().numpy(), q.cpu().numpy(), w.n)
+    assert_scores_close(s_nib.cpu().numpy(), o_scores, o_l1)
+    st_n = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, fixed_r=32, nibbles=nib)
+    st_p = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, fixed_r=32)
+    a = st_n.run(q)
+    b = st_p.run(q)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
