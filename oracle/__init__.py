@@ -52,6 +52,8 @@ def _lib():
         lib.orc_dequant_rows.argtypes = [P, P, I64, I, I64, I64, P, I64, P, I, P]
         lib.orc_calibrate.restype = I
         lib.orc_calibrate.argtypes = [P, I, I64, I64, I, I64, I64, P, P, P]
+        lib.orc_layer_budgets.restype = I
+        lib.orc_layer_budgets.argtypes = [P, P, I64, I, I, I, I64, P]
         lib.orc_pack_nibbles.restype = I
         lib.orc_pack_nibbles.argtypes = [P, I, I64, I64, I, I64, I64, P, I64]
         lib.orc_union_attention.restype = I
@@ -246,3 +248,15 @@ def pack_nibbles(keys: np.ndarray, nb_stride: int | None = None) -> np.ndarray:
     nib = np.zeros((H, D, 4, nbs), dtype=np.uint64)
     _check(_lib().orc_pack_nibbles(_ptr(keys), dt, H, n, D, n * D, D, _ptr(nib), nbs), "pack_nibbles")
     return nib
+
+
+def layer_budgets(sigma2: np.ndarray, q: np.ndarray, layers: int, total_bits: int) -> np.ndarray:
+    """Greedy per-layer split of ``total_bits`` plane bits: int32 [H], the
+    budget of each group (equal within a layer of H/layers groups)."""
+    sigma2 = np.ascontiguousarray(sigma2, dtype=np.float32)
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    H, G, D = q.shape
+    out = np.zeros(H, dtype=np.int32)
+    _check(_lib().orc_layer_budgets(_ptr(sigma2), _ptr(q), H, G, D, int(layers), int(total_bits), _ptr(out)),
+           "layer_budgets")
+    return out

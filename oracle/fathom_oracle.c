@@ -36,6 +36,9 @@
  *   orc_union_attention  softmax attention of each query head over its KV
  *                      head's union of winner rows (byte-accounting
  *                      section: the winner rows a step fetches)
+ *   orc_layer_budgets  greedy split of a total plane-bit budget across
+ *                      layers (water-filling section, per-layer plan
+ *                      paragraph)
  *   orc_pack_nibbles   the same 4-bit codes stored whole, 4 bits per token
  *                      (the fixed-depth scans' 4-bit coordinates of the
  *                      byte-accounting section), 16 tokens per 64-bit word
@@ -566,5 +569,64 @@ int orc_pack_nibbles(const void* keys, int key_dtype, int64_t H, int64_t n, int 
             }
         }
     }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-layer budgets (water-filling section: layers differ in how sharp  */
+/* their scores are, so a greedy pass on calibration data may give each  */
+/* layer its own budget; the default is the flat budget).                */
+/* The groups of layer l are h = l*P .. l*P + P - 1 (P = H / layers),    */
+/* and all get the layer's budget B_l.  A group's expected squared score */
+/* error under its plan is E_h(B) = sum_j w_j 4^-t_j, and reading the    */
+/* b-th largest item v (an item w_j 4^-t) lowers it by 3v/4.  The cost   */
+/* of layer l is its groups' error relative to their unread error,      */
+/*   C_l(B) = sum_h E_h(B) / N_l,   N_l = sum_h sum_j w_hj,              */
+/* so one more bit for every group of the layer gains                    */
+/*   g_l(b) = 0.75 * (sum_h v_h,(b)) / N_l,   b = B_l + 1,               */
+/* which does not grow with b.  The greedy gives the total budget one    */
+/* bit per step to the layer with the largest next gain (ties to the     */
+/* lower layer), at most 4D bits per layer.  Sums run in double, in the  */
+/* order written (h ascending, then j ascending).                        */
+/* ------------------------------------------------------------------ */
+int orc_layer_budgets(const float* sigma2, const float* q, int64_t H, int G, int D, int layers,
+                      int64_t total_bits, int32_t* budget_out)
+{
+    if (!sigma2 || !q || !budget_out || H <= 0 || G <= 0 || D <= 0 || layers <= 0 || H % layers) return ORC_EINVAL;
+    int64_t P = H / layers, NI = 4 * (int64_t)D;
+    double* items = (double*)calloc((size_t)(H * NI), sizeof(double));
+    double* N = (double*)calloc((size_t)layers, sizeof(double));
+    int64_t* ptr = (int64_t*)calloc((size_t)layers, sizeof(int64_t));
+    if (!items || !N || !ptr) { free(items); free(N); free(ptr); return ORC_ENOMEM; }
+    for (int64_t h = 0; h < H; ++h) {
+        double* it = items + h * NI;
+        int npos = 0;
+        for (int j = 0; j < D; ++j) {
+            float w = orc_importance(&sigma2[h * D + j], &q[(h * G) * D + j], G, D);
+            if (w > 0.0f) {
+                N[h / P] += (double)w;
+                for (int t = 0; t < 4; ++t) it[npos++] = ldexp((double)w, -2 * t);
+            }
+        }
+        qsort(it, (size_t)npos, sizeof(double), cmp_desc_double);   /* the rest stays 0 */
+    }
+    int64_t T = total_bits < 0 ? 0 : total_bits;
+    if (T > layers * NI) T = layers * NI;
+    for (int64_t step = 0; step < T; ++step) {
+        int best = -1;
+        double bg = 0.0;
+        for (int l = 0; l < layers; ++l) {
+            if (ptr[l] >= NI) continue;
+            double S = 0.0;
+            for (int64_t h = l * P; h < (l + 1) * P; ++h) S += items[h * NI + ptr[l]];
+            double g = N[l] > 0.0 ? 0.75 * S / N[l] : 0.0;
+            if (best < 0 || g > bg) { best = l; bg = g; }
+        }
+        ptr[best]++;
+    }
+    for (int64_t h = 0; h < H; ++h) budget_out[h] = (int32_t)ptr[h / P];
+    free(items);
+    free(N);
+    free(ptr);
     return ORC_OK;
 }

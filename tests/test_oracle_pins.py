@@ -613,3 +613,56 @@ def test_nibbles_hold_the_plane_codes(orc):
             codes = np.array([(int(nib[h, j, (i % 64) // 16, b]) >> (4 * (i % 16))) & 15 for j in range(D)])
             khat = (codes - 7.5) * s[h, :, b] / 8.0
             assert np.allclose(sc[h, :, i], q[h].astype(np.float64) @ khat, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Per-layer budgets (section 方法二, per-layer plan paragraph)
+# --------------------------------------------------------------------------
+def _layer_cost(orc, s2, q, layers, budgets):
+    """sum over layers of the layer's expected squared score error relative
+    to its unread error, from the oracle's own plans (fp64 over fp32 w)."""
+    H, G, D = q.shape
+    w = orc.importance(s2, q).astype(np.float64)
+    depth, _, _, _ = orc.plan(s2, q, np.asarray(budgets, np.int32))
+    E = (w * 4.0 ** (-depth.astype(np.float64))).sum(1)
+    P = H // layers
+    return sum(E[l * P:(l + 1) * P].sum() / w[l * P:(l + 1) * P].sum() for l in range(layers))
+
+
+def test_layer_budgets_are_optimal_by_brute_force(orc):
+    """On tiny layers (D = 2, 2 groups each) the greedy split reaches the
+    least total relative error over every split of the total, and it always
+    spends the whole total (capped at 4D per layer)."""
+    rng = np.random.default_rng(31)
+    for trial in range(12):
+        L, P, D, G = 3, 2, 2, 2
+        H = L * P
+        s2 = np.exp(rng.normal(0, 1.5, (H, D))).astype(np.float32)
+        q = rng.standard_normal((H, G, D)).astype(np.float32)
+        T = int(rng.integers(0, 4 * D * L + 3))
+        b = orc.layer_budgets(s2, q, L, T)
+        per_layer = b[::P]
+        assert np.array_equal(b, np.repeat(per_layer, P))
+        assert per_layer.sum() == min(T, 4 * D * L) and per_layer.max() <= 4 * D
+        best = min(_layer_cost(orc, s2, q, L, np.repeat(np.array(split), P))
+                   for split in itertools.product(range(4 * D + 1), repeat=L) if sum(split) == min(T, 4 * D * L))
+        assert _layer_cost(orc, s2, q, L, b) <= best * (1 + 1e-12)
+
+
+def test_layer_budgets_invariances(orc):
+    """Identical layers share the total evenly (the remainder to the lower
+    layers); scaling one layer's sigma^2 by a power of 4 leaves its relative
+    curve, so the split, unchanged; one layer gets the flat budget."""
+    rng = np.random.default_rng(32)
+    P, D, G = 2, 16, 4
+    s2 = np.exp(rng.normal(0, 1, (P, D))).astype(np.float32)
+    q = rng.standard_normal((P, G, D)).astype(np.float32)
+    s2_3, q_3 = np.tile(s2, (3, 1)), np.tile(q, (3, 1, 1))
+    assert list(orc.layer_budgets(s2_3, q_3, 3, 3 * 40 + 2)[::P]) == [41, 41, 40]
+    s2_a = np.exp(rng.normal(0, 1, (3 * P, D))).astype(np.float32)
+    q_a = rng.standard_normal((3 * P, G, D)).astype(np.float32)
+    base = orc.layer_budgets(s2_a, q_a, 3, 150)
+    s2_b = s2_a.copy()
+    s2_b[P:2 * P] *= np.float32(16.0)
+    assert np.array_equal(orc.layer_budgets(s2_b, q_a, 3, 150), base)
+    assert np.all(orc.layer_budgets(s2_a, q_a, 1, 50) == 50)
