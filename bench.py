@@ -542,6 +542,43 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     nrows = int(cnt.clamp(min=0).sum().item())
     out["reconstruct_union_rows"] = {"ms": tot / 5, "rows": nrows, "rows_per_s": nrows / (tot / 5 / 1e3),
                                      "out_GBps": nrows * w.D * 4 / (tot / 5 / 1e3) / 1e9}
+    # Per-layer budgets from the greedy split (mean 48 bits per group), on
+    # the step's own queries and on an independent draw of calibration
+    # queries, against the flat budget: step time and the relative expected
+    # score error sum_l (sum_h sum_j w 4^-t / sum_h sum_j w) on the step's queries.
+    from long_context_decode_bit_b200 import inputs as _inq
+    nl = w.H // 8 if w.H % 8 == 0 else 1
+    qf = q.float()
+    wimp = sigma2 * (qf * qf).sum(1)
+
+    def rel_err(budget):
+        dp, _, _, _ = fathom.plan(sigma2, q, budget)
+        e = (wimp.double() * torch.pow(4.0, -dp.double())).sum(1).view(nl, -1).sum(1)
+        return float((e / wimp.double().sum(1).view(nl, -1).sum(1)).sum().item())
+    q_cal = _inq.queries(dataclasses.replace(w, seed=w.seed + 1000), 0, w.H, device=device).float().contiguous()
+    lb = {"layers": nl, "rel_error_flat": rel_err(48)}
+    for tag, qc in (("in_sample", q), ("calibration_draw", q_cal)):
+        bud = fathom.layer_budgets(sigma2, qc, nl, nl * 48)
+        stl = fathom.Step(planes, scales, w.n, sigma2, w.G, k, budget=bud)
+
+        def onel(ev, st=stl):
+            st.run_plan(q)
+            st.run_prepare(q)
+            if ev is not None:
+                ev[0].record()
+            st.run_filter(q)
+            if ev is not None:
+                ev[1].record()
+            st.run_topk()
+        onel(None)
+        torch.cuda.synchronize(device)
+        fbl = stl.repair(q)
+        tot, fk = time_steps(onel, 5, 2, device, kernel_events=True)
+        bl = bud.view(nl, -1)[:, 0].tolist()
+        lb[tag] = {"ms_per_step": tot / 5, "scan_ms": statistics.fmean(fk), "budget_min": min(bl),
+                   "budget_max": max(bl), "rel_error": rel_err(bud), "fallback_groups": fbl}
+        del stl
+    out["per_layer_greedy_B48"] = lb
     # The fixed 136-bit scan over the nibble store (whole 4-bit codes): the
     # same bytes as the plane scan at depth 4, decoded from nibbles.
     nib = fathom.nibbles_from_planes(planes, w.n)

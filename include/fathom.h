@@ -188,6 +188,39 @@ int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D,
                 fathom_stream_t stream);
 
 /*
+ * fathom_layer_budgets_workspace_bytes -- scratch fathom_layer_budgets needs
+ * (HOST call); 0 for unsupported sizes.
+ */
+size_t fathom_layer_budgets_workspace_bytes(int64_t H, int D);
+
+/*
+ * fathom_layer_budgets -- per-layer plane-bit budgets from calibration
+ * queries (方法二, per-layer plan paragraph: layers differ in how sharp
+ * their scores are, and a greedy pass on calibration data can give each its
+ * own budget; the pages' default stays the flat budget).  The groups of
+ * layer l are h = l*P .. l*P + P - 1, P = H / layers, and all get B_l.
+ * With w_j the plan's importance (same fp32 order) and v_h,(b) the b-th
+ * largest item w_j 4^-t of group h, one more bit for layer l lowers its
+ * error relative to its unread error sum_h sum_j w_hj by
+ *   g_l(b) = 0.75 * sum_h v_h,(b) / sum_h sum_j w_hj.
+ * The greedy gives total_bits (capped at layers * 4D) one bit at a time to
+ * the layer with the largest next gain, ties to the lower layer, at most
+ * 4D per layer; sums run in double in a fixed order, so the result is
+ * defined bit for bit.  Pass budget_bits to fathom_plan.
+ *
+ *   sigma2, q   DEVICE, as for fathom_plan (q: calibration queries).
+ *   layers      1..1024, dividing H.
+ *   total_bits  the budget of all layers together (e.g. layers * 48).
+ *   budget_bits DEVICE out, int32 [H].
+ *   workspace, ws_bytes  DEVICE scratch of at least
+ *               fathom_layer_budgets_workspace_bytes(H, D) bytes, 256-byte
+ *               aligned.
+ */
+int fathom_layer_budgets(const float* sigma2, const float* q, int64_t H, int G, int D, int layers,
+                         int64_t total_bits, int32_t* budget_bits, void* workspace, size_t ws_bytes,
+                         fathom_stream_t stream);
+
+/*
  * fathom_plan_fixed -- a fixed-depth comparator plan: the r channels with
  * the largest a_j = |q_{0,j}| + |q_{1,j}| + ... + |q_{G-1,j}| (single
  * precision, that order; ties to the lower j) read at `bits` planes, the

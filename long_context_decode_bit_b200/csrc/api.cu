@@ -22,6 +22,9 @@ int launch_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t 
                         int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count, int bits,
                         float* out, cudaStream_t stream);
 
+size_t layer_budgets_workspace_bytes(int64_t H, int D);
+int launch_layer_budgets(const float* sigma2, const float* q, int64_t H, int G, int D, int layers, int64_t total_bits,
+                         int32_t* budget, void* ws, cudaStream_t stream);
 size_t calibrate_workspace_bytes(int64_t H, int D, bool with_cov);
 int launch_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t sh, int64_t st,
                      float* mean, float* sigma2, float* cov, void* ws, cudaStream_t stream);
@@ -188,6 +191,31 @@ int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, in
     FATHOM_TRY(check_device_ptr(scales));
     return launch_pack(keys, key_dtype, H, n, D, key_stride_h, key_stride_tok, planes, scales, nb_stride,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fathom_layer_budgets_workspace_bytes(int64_t H, int D)
+{
+    if (H <= 0 || !dims_ok(D, 1)) return 0;
+    return layer_budgets_workspace_bytes(H, D);
+}
+
+int fathom_layer_budgets(const float* sigma2, const float* q, int64_t H, int G, int D, int layers,
+                         int64_t total_bits, int32_t* budget_bits, void* workspace, size_t ws_bytes,
+                         fathom_stream_t stream)
+{
+    if (H < 0 || H > 0x7FFFFFFF || layers < 1 || layers > 1024 || total_bits < 0) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
+    if (H == 0) return FATHOM_OK;
+    if (H % layers) return FATHOM_ERR_INVALID_ARG;
+    if (ws_bytes < layer_budgets_workspace_bytes(H, D)) return FATHOM_ERR_WORKSPACE;
+    if (!aligned(sigma2, 4) || !aligned(q, 4) || !aligned(budget_bits, 4) || !aligned(workspace, 256))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(sigma2));
+    FATHOM_TRY(check_device_ptr(q));
+    FATHOM_TRY(check_device_ptr(budget_bits));
+    FATHOM_TRY(check_device_ptr(workspace));
+    return launch_layer_budgets(sigma2, q, H, G, D, layers, total_bits, budget_bits, workspace,
+                                reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fathom_calibrate_workspace_bytes(int64_t H, int D, int with_cov)

@@ -145,7 +145,117 @@ __global__ void plan_fixed_kernel(const float* __restrict__ q, int G, int D, int
     write_active(j, t, D, h, active, n_active, warp_cnt);
 }
 
+// Per-layer budgets, step 1 (one CTA per group, one thread per channel):
+// the group's items w_j 4^-t (w in the plan's fp32 order; 0 for a channel
+// whose w is not positive) sorted in descending order into items[h][4D],
+// and w itself (0 when not positive) into wout[h][D].
+__global__ void layer_items_kernel(const float* __restrict__ sigma2, const float* __restrict__ q, int G, int D,
+                                   int npow2, double* __restrict__ items, float* __restrict__ wout)
+{
+    __shared__ double it[4 * kMaxD];
+    const int64_t h = blockIdx.x;
+    const int j = threadIdx.x;   // blockDim.x == D
+    const float* qh = q + h * G * D + j;
+    float acc = __fmul_rn(qh[0], qh[0]);
+    for (int g = 1; g < G; ++g) acc = __fadd_rn(acc, __fmul_rn(qh[g * D], qh[g * D]));
+    const float w = __fmul_rn(sigma2[h * D + j], acc);
+    const bool pos = w > 0.0f;
+    wout[h * D + j] = pos ? w : 0.0f;
+    for (int t = 0; t < 4; ++t) it[4 * j + t] = pos ? ldexp(static_cast<double>(w), -2 * t) : 0.0;
+    for (int i = 4 * D + j; i < npow2; i += D) it[i] = -1.0;   // below every item
+    // bitonic sort, descending
+    for (int size = 2; size <= npow2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            __syncthreads();
+            for (int i = j; i < (npow2 >> 1); i += D) {
+                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const double x = it[lo], y = it[hi];
+                if (up ? (x < y) : (x > y)) { it[lo] = y; it[hi] = x; }
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = j; i < 4 * D; i += D) items[h * 4 * D + i] = it[i];
+}
+
+// Per-layer budgets, step 2 (one warp): the greedy.  Layer l (groups
+// l*P .. l*P+P-1) has the next gain g_l(b) = 0.75 * (sum_h items[h][b-1]) / N_l,
+// N_l = sum over its groups and channels of w; each step gives one bit to
+// the layer with the largest next gain, ties to the lower layer.  Sums run
+// in double in the order h ascending, then j ascending.
+__global__ void layer_greedy_kernel(const double* __restrict__ items, const float* __restrict__ w, int64_t H, int D,
+                                    int layers, int64_t T, int32_t* __restrict__ budget)
+{
+    extern __shared__ __align__(8) unsigned char lsm[];
+    double* N = reinterpret_cast<double*>(lsm);
+    double* gain = N + layers;
+    int* ptr = reinterpret_cast<int*>(gain + layers);
+    const int lane = threadIdx.x;
+    const int64_t P = H / layers;
+    const int NI = 4 * D;
+    auto next_gain = [&](int l, int b) -> double {   // gain of the layer's (b+1)-th bit
+        double S = 0.0;
+        for (int64_t h = l * P; h < (l + 1) * P; ++h) S += items[h * NI + b];
+        return N[l] > 0.0 ? 0.75 * S / N[l] : 0.0;
+    };
+    for (int l = lane; l < layers; l += 32) {
+        double n = 0.0;
+        for (int64_t h = l * P; h < (l + 1) * P; ++h)
+            for (int j = 0; j < D; ++j) n += static_cast<double>(w[h * D + j]);
+        N[l] = n;
+        ptr[l] = 0;
+        gain[l] = next_gain(l, 0);
+    }
+    __syncwarp();
+    for (int64_t step = 0; step < T; ++step) {
+        double bg = -1.0;
+        int bl = INT32_MAX;
+        for (int l = lane; l < layers; l += 32) {
+            if (ptr[l] >= NI) continue;
+            if (gain[l] > bg) { bg = gain[l]; bl = l; }   // ascending l: the first maximum wins
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double og = __shfl_xor_sync(0xffffffffu, bg, o);
+            const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
+            if (og > bg || (og == bg && ol < bl)) { bg = og; bl = ol; }
+        }
+        if (bl == INT32_MAX) break;   // every layer full (T was capped before the launch)
+        if ((bl & 31) == lane) {
+            const int b = ++ptr[bl];
+            gain[bl] = b < NI ? next_gain(bl, b) : 0.0;
+        }
+        __syncwarp();
+    }
+    for (int64_t h = lane; h < H; h += 32) budget[h] = ptr[h / P];
+}
+
 }  // namespace
+
+size_t layer_budgets_workspace_bytes(int64_t H, int D)
+{
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    return up(sizeof(double) * H * 4 * D) + up(sizeof(float) * H * D);
+}
+
+int launch_layer_budgets(const float* sigma2, const float* q, int64_t H, int G, int D, int layers, int64_t total_bits,
+                         int32_t* budget, void* ws, cudaStream_t stream)
+{
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    double* items = static_cast<double*>(ws);
+    float* w = reinterpret_cast<float*>(static_cast<char*>(ws) + up(sizeof(double) * H * 4 * D));
+    int npow2 = 1;
+    while (npow2 < 4 * D) npow2 <<= 1;
+    layer_items_kernel<<<static_cast<unsigned>(H), D, 0, stream>>>(sigma2, q, G, D, npow2, items, w);
+    int st = launch_status();
+    if (st) return st;
+    int64_t T = total_bits < 0 ? 0 : total_bits;
+    if (T > static_cast<int64_t>(layers) * 4 * D) T = static_cast<int64_t>(layers) * 4 * D;
+    const size_t smem = sizeof(double) * 2 * layers + sizeof(int) * layers;
+    layer_greedy_kernel<<<1, 32, smem, stream>>>(items, w, H, D, layers, T, budget);
+    return launch_status();
+}
 
 int launch_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,
                 int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,

@@ -39,7 +39,8 @@ EXPORTS = (
     "fathom_topk_workspace_bytes", "fathom_topk", "fathom_dequant_rows", "fathom_scan_topk_noalloc",
     "fathom_device_status", "fathom_calibrate_workspace_bytes", "fathom_calibrate",
     "fathom_union_attention_workspace_bytes", "fathom_union_attention",
-    "fathom_nibbles_from_planes", "fathom_scan_nibbles",
+    "fathom_nibbles_from_planes", "fathom_scan_nibbles", "fathom_layer_budgets_workspace_bytes",
+    "fathom_layer_budgets",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -87,6 +88,8 @@ def load(path: str | None = None):
         "fathom_calibrate": (I, [P, I, I64, I64, I, I64, I64, P, P, P, P, SZ, P]),
         "fathom_union_attention_workspace_bytes": (SZ, [I64, I, I, I64]),
         "fathom_nibbles_from_planes": (I, [P, I64, I, I64, I64, P, P]),
+        "fathom_layer_budgets_workspace_bytes": (SZ, [I64, I]),
+        "fathom_layer_budgets": (I, [P, P, I64, I, I, I, I64, P, P, SZ, P]),
         "fathom_scan_nibbles": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, SZ, I, P]),
         "fathom_union_attention": (I, [P, P, I, I64, I64, I, I64, I64, P, I, P, P, I64, ctypes.c_float, P, P, SZ, P]),
     }
@@ -181,6 +184,19 @@ def plan(sigma2: torch.Tensor, q: torch.Tensor, budget, out=None, stream=None):
     _check(lib().fathom_plan(_p(sigma2), _p(q), H, G, D, bptr, flat, _p(depth), _p(active), _p(n_active),
                              _p(theta), _stream(stream)), "fathom_plan")
     return depth, active, n_active, theta
+
+
+def layer_budgets(sigma2: torch.Tensor, q: torch.Tensor, layers: int, total_bits: int, out=None, stream=None):
+    """Greedy per-layer split of ``total_bits`` plane bits from calibration
+    queries q [H][G][D]: int32 [H] budgets for ``plan``."""
+    H, G, D = q.shape
+    dev = q.device
+    if out is None:
+        out = torch.empty(H, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(int(lib().fathom_layer_budgets_workspace_bytes(H, D)), 1), dtype=torch.uint8, device=dev)
+    _check(lib().fathom_layer_budgets(_p(sigma2), _p(q), H, G, D, int(layers), int(total_bits), _p(out), _p(ws),
+                                      ws.numel(), _stream(stream)), "fathom_layer_budgets")
+    return out
 
 
 def plan_fixed(q: torch.Tensor, r: int, out=None, stream=None, bits: int = 4):

@@ -92,6 +92,11 @@ def test_rejections_before_any_cuda_call(lib):
     assert lib.fathom_scan_nibbles(n, n, 1, 100, 100, 2, n, n, n, 4, 0, n, n, 0, 1, n) == fathom.ERR_UNSUPPORTED
     assert lib.fathom_nibbles_from_planes(n, 1, 48, 100, 2, n, n) == fathom.ERR_UNSUPPORTED
     assert lib.fathom_nibbles_from_planes(n, 1, 128, 1000, 15, n, n) == fathom.ERR_INVALID_ARG   # stride < nb
+    assert lib.fathom_layer_budgets_workspace_bytes(288, 128) == 288 * 512 * 8 + 288 * 128 * 4
+    assert lib.fathom_layer_budgets(n, n, 10, 4, 128, 3, 100, n, n, 0, n) == fathom.ERR_INVALID_ARG   # 3 does not divide 10
+    assert lib.fathom_layer_budgets(n, n, 10, 4, 128, 0, 100, n, n, 0, n) == fathom.ERR_INVALID_ARG   # no layer
+    assert lib.fathom_layer_budgets(n, n, 10, 4, 100, 5, 100, n, n, 0, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_layer_budgets(fake, fake, 10, 4, 128, 5, 100, fake, fake, 64, n) == fathom.ERR_WORKSPACE
     ua = lib.fathom_union_attention
     assert ua(n, n, 0, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 0, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # M = 0
     assert ua(n, n, 2, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 8, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # dtype

@@ -454,3 +454,26 @@ def test_nibbles_bit_exact_and_scan_equals_full_depth(fathom_gpu, orc, w):
     b = st_p.run(q)
     torch.cuda.synchronize()
     assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+# --------------------------------------------------------------------------
+# Per-layer budgets (方法二, per-layer plan paragraph)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("w,layers,mean_bits", [
+    (dataclasses.replace(inputs.STEP_128K, name="lb-qwen", n=4096, n_cal=4096), 36, 48),
+    (dataclasses.replace(inputs.STEP_1M_LLAMA, name="lb-llama", H=64, n=4096, n_cal=4096), 8, 48),
+    (dataclasses.replace(inputs.TINY, name="lb-gauss", H=6, n=1024, n_cal=1024), 3, 200)],
+    ids=["qwen-36-layers", "llama-8-layers", "gauss-3-layers-capped"])
+def test_layer_budgets_match_oracle(fathom_gpu, orc, w, layers, mean_bits):
+    """The greedy split equals the oracle's integer for integer, spends the
+    whole total (capped at 4D per layer), and the plans it feeds respect it."""
+    k, q, s2 = make(w)
+    b = fathom_gpu.layer_budgets(s2, q, layers, layers * mean_bits)
+    torch.cuda.synchronize()
+    ref = orc.layer_budgets(s2.cpu().numpy(), q.cpu().numpy(), layers, layers * mean_bits)
+    got = b.cpu().numpy()
+    assert np.array_equal(got, ref)
+    per = got.reshape(layers, -1)
+    assert np.all(per == per[:, :1]) and per[:, 0].sum() == min(layers * mean_bits, layers * 4 * w.D)
+    depth, _, _, _ = fathom_gpu.plan(s2, q, b)
+    assert np.all(depth.int().sum(1).cpu().numpy() <= got)
