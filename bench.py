@@ -623,6 +623,33 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     out["union_attention_one_layer"] = {"groups": la, "ms": tot / 5, "rows": arows,
                                         "kv_bytes": arows * 2 * w.D * kc.element_size(),
                                         "kv_GBps": arows * 2 * w.D * kc.element_size() / (tot / 5 / 1e3) / 1e9}
+    # The same kernel across a whole step's 288 groups: a 131,072-key K/V
+    # cache per group and 2,048 scattered union rows each (random, sorted).
+    aw = dataclasses.replace(w, name="attention-288x131072", n=131072, seed=w.seed + 7)
+    try:
+        kc2 = _inp.keys(aw, 0, aw.H, device=device)
+        vc2 = _inp.values(aw, 0, aw.H, device=device)
+        gen = torch.Generator(device=device)
+        gen.manual_seed(97)
+        M2 = w.G * k
+        uni2 = torch.sort(torch.randperm(aw.n, generator=gen, device=device)[:M2].repeat(aw.H, 1), dim=1)[0]
+        uni2 = uni2.to(torch.int32).contiguous()
+        cnt2 = torch.full((aw.H,), M2, dtype=torch.int32, device=device)
+        out2 = torch.empty((aw.H, w.G, w.D), dtype=torch.float32, device=device)
+        ws2 = torch.empty(fathom.union_attention_workspace_bytes(aw.H, w.G, w.D, M2), dtype=torch.uint8, device=device)
+
+        q2 = q.float().contiguous()
+
+        def att2(ev):
+            fathom.union_attention(kc2, vc2, q2, uni2, cnt2, out=out2, workspace=ws2)
+        att2(None)
+        tot, _ = time_steps(att2, 5, 2, device)
+        nb2 = aw.H * M2 * 2 * w.D * kc2.element_size()
+        out["union_attention_288_groups"] = {"groups": aw.H, "n": aw.n, "rows_per_group": M2, "ms": tot / 5,
+                                             "kv_bytes": nb2, "kv_GBps": nb2 / (tot / 5 / 1e3) / 1e9}
+        del kc2, vc2, uni2, cnt2, out2, ws2, q2
+    except torch.cuda.OutOfMemoryError:
+        out["union_attention_288_groups"] = "skipped: not enough device memory"
     del st, rows_out, kc, vc, att_out, att_ws
     # Session calibration from the session's own keys: one layer's 8 KV heads
     # and one KV head at n = 100,000, with and without the covariance.

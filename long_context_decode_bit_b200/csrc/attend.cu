@@ -9,9 +9,10 @@
 //
 // Layout (split over the union, as in split-K decoding): a CTA takes a
 // chunk of up to kAttRows union rows of one group.
-//   1. Warp w scores rows w, w+8, ...: lane l reads channels l, l+32, ...
-//      of the row (64-byte coalesced pieces), keeps G partial dots and
-//      reduces them across the warp with butterfly shuffles.
+//   1. Warp w scores its rows four at a time (all four rows' loads issued
+//      before the arithmetic): lane l reads channels l, l+32, ... of a row
+//      (64-byte coalesced pieces), keeps G partial dots and reduces them
+//      across the warp with butterfly shuffles.
 //   2. Warp g turns head g's chunk scores into exp(s - m_g) and their sum.
 //   3. Thread t accumulates channel t % D over the rows of its slice
 //      (t / D) for all G heads; the slices are summed in shared memory.
@@ -77,27 +78,40 @@ attend_chunk_kernel(const AttArgs a)
     }
     __syncthreads();
 
-    // 1. scores
-    for (int r = warp; r < rows; r += kAttThreads / 32) {
-        const int i = rowi[r];
-        float dot[G];
+    // 1. scores: each warp takes kAttBatch rows at a time and issues all
+    // their loads before the arithmetic, so that several rows are in flight.
+    constexpr int kAttBatch = 4;
+    const int chunks_d = D / 32;   // channels per lane
+    for (int r0w = warp * kAttBatch; r0w < rows; r0w += (kAttThreads / 32) * kAttBatch) {
+        float kv[kAttBatch][kMaxD / 32];
 #pragma unroll
-        for (int g = 0; g < G; ++g) dot[g] = 0.0f;
-        if (i >= 0) {
-            const int64_t base = h * a.sh + static_cast<int64_t>(i) * a.st;
-            for (int ch = lane; ch < D; ch += 32) {
-                const float kv = kv_at<DT>(a.k, base + ch);
+        for (int b = 0; b < kAttBatch; ++b) {
+            const int r = r0w + b;
+            const int i = r < rows ? rowi[r] : -1;
+            const int64_t base = h * a.sh + static_cast<int64_t>(i < 0 ? 0 : i) * a.st;
 #pragma unroll
-                for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g * D + ch], kv, dot[g]);
-            }
+            for (int cc = 0; cc < kMaxD / 32; ++cc)
+                kv[b][cc] = (i >= 0 && cc < chunks_d) ? kv_at<DT>(a.k, base + lane + 32 * cc) : 0.0f;
         }
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+        for (int b = 0; b < kAttBatch; ++b) {
+            const int r = r0w + b;
+            float dot[G];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) dot[g] += __shfl_xor_sync(kFullMask, dot[g], o);
-        if (lane == 0)
+            for (int g = 0; g < G; ++g) dot[g] = 0.0f;
 #pragma unroll
-            for (int g = 0; g < G; ++g) sc[g * kAttRows + r] = i >= 0 ? dot[g] : -INFINITY;
+            for (int cc = 0; cc < kMaxD / 32; ++cc)
+                if (cc < chunks_d)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) dot[g] = fmaf(qs[g * D + lane + 32 * cc], kv[b][cc], dot[g]);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) dot[g] += __shfl_xor_sync(kFullMask, dot[g], o);
+            if (lane == 0 && r < rows)
+#pragma unroll
+                for (int g = 0; g < G; ++g) sc[g * kAttRows + r] = rowi[r] >= 0 ? dot[g] : -INFINITY;
+        }
     }
     __syncthreads();
 
@@ -130,10 +144,10 @@ attend_chunk_kernel(const AttArgs a)
         float acc[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) acc[g] = 0.0f;
+#pragma unroll 8
         for (int r = sl; r < rows; r += slices) {
             const int i = rowi[r];
-            if (i < 0) continue;
-            const float vv = kv_at<DT>(a.v, h * a.sh + static_cast<int64_t>(i) * a.st + d);
+            const float vv = i >= 0 ? kv_at<DT>(a.v, h * a.sh + static_cast<int64_t>(i) * a.st + d) : 0.0f;
 #pragma unroll
             for (int g = 0; g < G; ++g) acc[g] = fmaf(sc[g * kAttRows + r], vv, acc[g]);
         }
