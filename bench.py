@@ -361,7 +361,7 @@ def run_gpu(args):
     d2h = sum(t.numel() * t.element_size() for t in res_host)
 
     sweep = None
-    if not args.no_sweep:
+    if not args.no_sweep and world == 1:   # the sweep is a single-GPU report; scaling runs time the step only
         sweep = run_sweep(w, planes, scales, sigma2, q, k, device, log)
 
     result = {
