@@ -637,8 +637,8 @@ CandLayout cand_layout(int64_t H, int G, int64_t n, int k)
         L.n_sample = 0;
         L.m_rank = 0;
     } else {
-        int64_t S = k / 16;
-        S = S < 1 ? 1 : (S > 32 ? 32 : S);
+        int64_t S = k / 8;
+        S = S < 1 ? 1 : (S > 64 ? 64 : S);
         if (S > L.tiles / 2) S = L.tiles / 2 < 1 ? 1 : L.tiles / 2;
         L.tile_stride = S;
         L.sample_tiles = ceil_div(L.tiles, S);

@@ -51,8 +51,9 @@ def test_host_only_entry_points(lib):
     assert small >= 2 * 4 * (16 + 1000 * 8)
     big = lib.fathom_scan_cand_bytes(288, 4, 2 ** 20, 512)
     # 1152 heads x (16384 survivor slots of 8 B, i.e. 8x the ~2048 expected,
-    # spread over the tiles + one count per tile + 32768 sample scores of 4 B)
-    per_head = 16384 * 8 + 32768 * 4
+    # spread over the tiles + one count per tile + 16384 sample scores of 4 B:
+    # 1 tile in 64 is sampled)
+    per_head = 16384 * 8 + 16384 * 4
     assert 1152 * per_head <= big < 1152 * (per_head + 4096 + 16) + 4 * 256
     # calibration scratch: two fp64 sums per (group, channel), plus the
     # fp64 D x D sums with the covariance
