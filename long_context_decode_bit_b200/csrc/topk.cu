@@ -19,6 +19,7 @@ namespace fathom {
 namespace {
 
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkCandThreads = 512;   // candidate lists are short: smaller CTAs, more of them per SM
 constexpr int kRadixBins = 2048;
 constexpr int kMaxTies = 4096;
 constexpr unsigned kFull = 0xffffffffu;
@@ -174,6 +175,7 @@ struct TopkArgs {
     int64_t cap, tiles, tslot;
     int64_t n;
     int k, kpow2;
+    int gather_cap;             // survivors gathered into shared memory (tile slots)
     int32_t* idx;               // [H*G][k]
 };
 
@@ -184,7 +186,7 @@ topk_kernel(const TopkArgs a)
     uint64_t* win = reinterpret_cast<uint64_t*>(smem);                        // kpow2
     int32_t* ties = reinterpret_cast<int32_t*>(win + a.kpow2);               // kMaxTies
     uint32_t* hist = reinterpret_cast<uint32_t*>(ties + kMaxTies);           // kRadixBins
-    int2* gathered = reinterpret_cast<int2*>(hist + kRadixBins);             // kCandGather (tile slots)
+    int2* gathered = reinterpret_cast<int2*>(hist + kRadixBins);             // gather_cap (tile slots)
     __shared__ uint32_t sh[2];
     __shared__ int w_cnt, t_cnt, warp_eq[kTopkThreads / 32], g_cnt, g_bad;
 
@@ -217,12 +219,12 @@ topk_kernel(const TopkArgs a)
             if (c <= 0) continue;
             if (c > a.tslot) { g_bad = 1; continue; }       // slot overflowed: keys were dropped
             const int base = atomicAdd(&g_cnt, c);
-            if (base + c > kCandGather) { g_bad = 1; continue; }
+            if (base + c > a.gather_cap) { g_bad = 1; continue; }
             for (int e = 0; e < c; ++e) gathered[base + e] = src[t * a.tslot + e];
         }
         __syncthreads();
         count = g_cnt;
-        if (g_bad || count < k || count > kCandGather) {   // could not prove exactness
+        if (g_bad || count < k || count > a.gather_cap) {   // could not prove exactness
             for (int r = tid; r < k; r += blockDim.x) out[r] = -1;
             return;
         }
@@ -355,10 +357,14 @@ int launch_tau(const float* sample, CandHeader* hdr, int64_t heads, int64_t n_sa
     return launch_status();
 }
 
+// Survivors one top-k CTA gathers: 8k, twice the ~4k a candidate pass keeps
+// (kCandGather at the largest k); more marks the group for the dense rerun.
+int gather_cap(int k) { return 8 * k < kCandGather ? 8 * k : kCandGather; }
+
 size_t topk_smem_bytes(int k, bool gather)
 {
     return sizeof(uint64_t) * pow2_at_least(k) + sizeof(int32_t) * kMaxTies + sizeof(uint32_t) * kRadixBins +
-           (gather ? sizeof(int2) * kCandGather : 0);
+           (gather ? sizeof(int2) * gather_cap(k) : 0);
 }
 
 int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
@@ -369,6 +375,7 @@ int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
     a.n = n;
     a.k = k;
     a.kpow2 = pow2_at_least(k);
+    a.gather_cap = gather_cap(k);
     a.idx = idx;
     bool gather = false;
     if (!scores) {
@@ -386,7 +393,9 @@ int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_status(e);
-    topk_kernel<<<dim3(G, static_cast<unsigned>(H)), kTopkThreads, smem, stream>>>(a);
+    // The dense path's index-ordered pass counts per warp over kTopkThreads
+    // threads; candidate lists take smaller CTAs.
+    topk_kernel<<<dim3(G, static_cast<unsigned>(H)), scores ? kTopkThreads : kTopkCandThreads, smem, stream>>>(a);
     int st = launch_status();
     if (st) return st;
     int32_t* fault = nullptr;
