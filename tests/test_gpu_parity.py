@@ -303,8 +303,9 @@ def test_append_repacks_the_tail_block(fathom_gpu, orc):
 @pytest.mark.parametrize("w,n", [(inputs.TINY, None), (inputs.TINY, 1024),
                                  (dataclasses.replace(inputs.LAYER_32K, name="cal", H=3, n=9000, seed=12), None),
                                  (dataclasses.replace(inputs.TINY, name="cal-d64", H=2, D=64, n=777, seed=13), None),
-                                 (dataclasses.replace(inputs.STEP_1M_LLAMA, name="cal-corr", H=2, n=5000, seed=14), None)],
-                         ids=["tiny", "tiny-first-1024", "qk-bf16-9000", "d64-ragged", "corr-bf16-5000"])
+                                 (dataclasses.replace(inputs.STEP_1M_LLAMA, name="cal-corr", H=2, n=5000, seed=14), None),
+                                 (dataclasses.replace(inputs.TINY, name="cal-d256", H=1, D=256, n=1500, seed=18), None)],
+                         ids=["tiny", "tiny-first-1024", "qk-bf16-9000", "d64-ragged", "corr-bf16-5000", "d256"])
 def test_calibrate_matches_oracle(fathom_gpu, orc, w, n):
     """Mean and sigma^2 equal the oracle's fp64 values rounded to fp32 (a
     one-ulp allowance covers the fp64 summation order); the covariance is
@@ -477,3 +478,39 @@ def test_layer_budgets_match_oracle(fathom_gpu, orc, w, layers, mean_bits):
     assert np.all(per == per[:, :1]) and per[:, 0].sum() == min(layers * mean_bits, layers * 4 * w.D)
     depth, _, _, _ = fathom_gpu.plan(s2, q, b)
     assert np.all(depth.int().sum(1).cpu().numpy() <= got)
+
+
+@pytest.mark.parametrize("D,G", [(64, 3), (256, 8), (32, 1)])
+def test_union_attention_other_shapes(fathom_gpu, orc, D, G):
+    """Odd and extreme head counts and head dims (fp32 cache), one chunk and
+    several, against the oracle with the same per-element bound."""
+    w = dataclasses.replace(inputs.TINY, name=f"att-{D}-{G}", H=2, n=2000, D=D, G=G, seed=19 + D + G)
+    k = inputs.keys(w, 0, w.H, device=DEV)
+    v = inputs.values(w, 0, w.H, device=DEV)
+    q = inputs.queries(w, 0, w.H, device=DEV).float().contiguous()
+    g = np.random.default_rng(D + G)
+    cnt = np.array([300, 1], np.int32)
+    uni = np.full((w.H, 300), -1, np.int32)
+    for h in range(w.H):
+        uni[h, :cnt[h]] = np.sort(g.choice(w.n, cnt[h], replace=False))
+    out = fathom_gpu.union_attention(k, v, q, torch.from_numpy(uni).to(DEV), torch.from_numpy(cnt).to(DEV))
+    torch.cuda.synchronize()
+    ref = orc.union_attention(_as_np(k), _as_np(v), _as_np(q), uni, cnt)
+    tol = _attention_tolerance(_as_np(k), _as_np(v), _as_np(q), uni, cnt)
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= tol + 1e-30), np.max(np.abs(got - ref) - tol)
+
+
+@pytest.mark.parametrize("D,G", [(64, 3), (256, 8)])
+def test_nibble_scan_other_shapes(fathom_gpu, orc, D, G):
+    """The nibble-store scan equals the full-depth plane scan bit for bit for
+    odd G (padded coefficient records) and the largest D and G."""
+    w = dataclasses.replace(inputs.TINY, name=f"nib-{D}-{G}", H=2, n=3001, D=D, G=G, seed=23 + D)
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    nib = fathom_gpu.nibbles_from_planes(planes, w.n)
+    depth, active, na = fathom_gpu.plan_fixed(q, D // 4)
+    s_nib = fathom_gpu.scan(nib, scales, w.n, active, na, q, nibbles=True)
+    s_pl = fathom_gpu.scan(planes, scales, w.n, active, na, q)
+    torch.cuda.synchronize()
+    assert torch.equal(s_nib, s_pl)
