@@ -601,8 +601,10 @@ int launch_scan_g(ScanArgs a, int64_t ltiles, unsigned H, cudaStream_t stream)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t slots = static_cast<int64_t>(sms) * scan_min_ctas<G>() * FATHOM_SCAN_WAVES;
-    const int64_t per = ceil_div(ltiles * static_cast<int64_t>(H), slots);
-    a.tiles_per_cta = static_cast<int>(per < 1 ? 1 : (per > FATHOM_SCAN_TILES_CAP ? FATHOM_SCAN_TILES_CAP : per));
+    int64_t per = ceil_div(ltiles * static_cast<int64_t>(H), slots);
+    per = per < 1 ? 1 : (per > FATHOM_SCAN_TILES_CAP ? FATHOM_SCAN_TILES_CAP : per);
+    per = ceil_div(ltiles, ceil_div(ltiles, per));   // the same CTAs per group, their tiles evened out
+    a.tiles_per_cta = static_cast<int>(per);
     const unsigned gx = static_cast<unsigned>(ceil_div(ltiles, a.tiles_per_cta));
     scan_kernel<G, NIB><<<dim3(gx, H), kScanThreads, smem, stream>>>(a);
     return launch_status();
