@@ -11,8 +11,10 @@
  *
  * Conventions for every entry point
  *   - Memory is owned by the caller.  The library never allocates, never
- *     frees and keeps no state between calls (except the per-thread last
- *     CUDA error code).  Pointers marked DEVICE must be readable (or
+ *     frees and keeps no state between calls, except the per-thread last
+ *     CUDA error code, one fault word per device (fathom_device_status) and
+ *     the fixed scratch array of fathom_scan_topk_noalloc, both static
+ *     device objects of the library.  Pointers marked DEVICE must be readable (or
  *     writable) by the current CUDA device: device memory, managed memory,
  *     or, where stated, page-locked host memory mapped into the device's
  *     address space.  Pointers marked HOST are ordinary host memory.
