@@ -35,6 +35,33 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(raw, name), name
 
 
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """A C11 program (no C++, -Wall -Wextra -pedantic -Werror) includes the
+    header, takes the address of every declared function and links against
+    the library; it then runs the host-only calls (no GPU needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = declared_functions()
+    src = ["#include \"fathom.h\"", "#include <stdio.h>", "int main(void) {",
+           "    void (*table[])(void) = {"]
+    src += [f"        (void (*)(void)){n}," for n in names]
+    src += ["    };",
+            "    printf(\"%d %u %s %lld\\n\", fathom_version(), (unsigned)(sizeof table / sizeof table[0]),",
+            "           fathom_status_string(FATHOM_ERR_OVERFLOW), (long long)fathom_nb_stride(1025));",
+            "    return table[0] == 0;", "}"]
+    c_file = tmp_path / "abi.c"
+    c_file.write_text("\n".join(src) + "\n")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(fathom.LIB_PATH)
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(c_file), "-L", libdir, "-lfathom", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[0] == "10000" and int(out[1]) == len(names) and out[-1] == "32"
+
+
 def test_host_only_entry_points(lib):
     assert lib.fathom_version() == 10000
     assert lib.fathom_status_string(0) == b"ok"
