@@ -567,6 +567,15 @@ def test_union_attention_special_cases(orc):
     a = orc.union_attention(k, v, q, rows, np.full(H, 40, np.int32))
     b = orc.union_attention(k, v, q, rows[:, ::-1].copy(), np.full(H, 40, np.int32))
     assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
+    # a very sharp query: the softmax collapses onto the best row of the
+    # union (its score exceeds the next by far more than 1), with no overflow
+    big = (q * np.float32(1e4)).astype(np.float32)
+    sharp = orc.union_attention(k, v, big, rows, np.full(H, 40, np.int32))
+    for h in range(H):
+        s_h = big[h].astype(np.float64) @ k[h, rows[h]].astype(np.float64).T
+        best = rows[h][np.argmax(s_h, axis=1)]
+        assert np.all(np.isfinite(sharp[h]))
+        assert np.allclose(sharp[h], v[h, best].astype(np.float64), rtol=1e-9, atol=1e-9)
     pad = np.concatenate([rows, np.full((H, 10), -1, np.int32)], axis=1)   # -1 padded past the count
     assert np.array_equal(orc.union_attention(k, v, q, pad, np.full(H, 40, np.int32)), a)
     assert not np.any(orc.union_attention(k, v, q, pad, np.array([0, -6], np.int32)))
