@@ -391,7 +391,6 @@ class Step:
         self.topk_out = (torch.empty((H, G, k), dtype=torch.int32, device=dev),
                          torch.empty((H, G * k), dtype=torch.int32, device=dev),
                          torch.empty(H, dtype=torch.int32, device=dev))
-        self.launches = 0
 
     def run_plan(self, q):
         if self.fixed_r is None:
