@@ -43,6 +43,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "ring.cuh"
 
 namespace fathom {
 
@@ -69,9 +70,6 @@ constexpr int kMaxTilesPerCta = FATHOM_SCAN_TILES_CAP;
 
 // Named barrier among the consumer warps (0 is __syncthreads).
 constexpr int kBarConsumers = 1;
-// Upper bound on the polls of one ring wait; a wait that runs out marks the
-// launch faulty and the warp leaves its loop instead of spinning for ever.
-constexpr int kSpinLimit = 1 << 22;
 
 enum ScanMode { kDense = 0, kSample = 1, kCandidate = 2 };
 
@@ -122,58 +120,6 @@ struct SharedScan {
     __align__(8) uint64_t full[kStages];   // ring: data of the stage has landed (32 producer lanes)
     __align__(8) uint64_t empty[kStages];  // ring: every consumer warp is done with the stage
 };
-
-// Named barriers with compile-time ids (a run-time id reserves all 16).
-template <int ID, int COUNT>
-__device__ __forceinline__ void bar_sync()
-{
-    asm volatile("bar.sync %0, %1;\n" ::"n"(ID), "n"(COUNT) : "memory");
-}
-
-template <int ID, int COUNT>
-__device__ __forceinline__ void bar_arrive()
-{
-    asm volatile("bar.arrive %0, %1;\n" ::"n"(ID), "n"(COUNT) : "memory");
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, int count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar) : "memory");
-}
-
-// One arrival on `bar` once every cp.async this thread has issued so far has landed.
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
-}
-
-// Wait for the phase of `bar` with the given parity to complete; false if
-// the poll limit ran out first.  Each poll suspends the thread for at most
-// about a microsecond, so a wait gives up after a few seconds at most.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
-{
-    for (int it = 0; it < kSpinLimit; ++it) {
-        uint32_t ok;
-        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-                     : "=r"(ok) : "r"(bar), "r"(parity), "n"(1000) : "memory");
-        if (ok) return true;
-    }
-    return false;
-}
-
-// 16-byte copy of which only the first `bytes` (0..16) are read; the rest is zero-filled.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int bytes)
-{
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 // Depth-1 values of the four tokens of one 32-bit half: +-1.0f.
 __device__ __forceinline__ void values_depth1(uint32_t w, int l, float (&v)[4])
