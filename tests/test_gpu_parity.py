@@ -325,17 +325,24 @@ def test_calibrate_matches_oracle(fathom_gpu, orc, w, n):
 
 def test_calibrate_sigma2_feeds_the_plan(fathom_gpu, orc):
     """sigma^2 from the calibration call over the first n_cal keys gives the
-    same plan as the harness statistic, bit for bit."""
+    same plan as the harness statistic, bit for bit, on every group whose
+    sigma^2 row came out identical; a group whose row differs (a one-ulp fp64
+    summation-order case) still gets the oracle's plan of its own sigma^2."""
     w = inputs.LAYER_32K
     k, q, s2 = make(w)
     _, s2_gpu, _ = fathom_gpu.calibrate(k, n=w.n_cal, with_mean=False)
     d_ref, a_ref, n_ref, _ = fathom_gpu.plan(s2, q, 48)
     d_cal, a_cal, n_cal, _ = fathom_gpu.plan(s2_gpu, q, 48)
     torch.cuda.synchronize()
-    diff = (s2_gpu != s2).sum().item()
-    assert diff <= 2   # one-ulp fp64 summation-order cases at most
-    if diff == 0:
-        assert torch.equal(d_ref, d_cal) and torch.equal(a_ref, a_cal) and torch.equal(n_ref, n_cal)
+    same = torch.all(s2_gpu == s2, dim=1).cpu().numpy()
+    assert (s2_gpu != s2).sum().item() <= 2   # one-ulp fp64 summation-order cases at most
+    for h in range(w.H):
+        if same[h]:
+            assert torch.equal(d_ref[h], d_cal[h]) and torch.equal(a_ref[h], a_cal[h]) and n_ref[h] == n_cal[h]
+        else:
+            d_o, a_o, n_o, _ = orc.plan(s2_gpu[h:h + 1].cpu().numpy(), q[h:h + 1].cpu().numpy(), 48)
+            assert np.array_equal(d_cal[h:h + 1].cpu().numpy(), d_o)
+            assert np.array_equal(np_u16(a_cal[h:h + 1]), a_o) and n_cal[h].item() == n_o[0]
 
 
 # --------------------------------------------------------------------------

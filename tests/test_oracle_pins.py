@@ -221,6 +221,51 @@ def test_importance_single_precision_order(orc):
     assert np.array_equal(w.view(np.uint32), want.view(np.uint32))
 
 
+def test_importance_is_each_channels_measured_score_error(orc):
+    """The importance w_j = sigma_j^2 sum_g q_{g,j}^2 is what a channel's
+    unread or partly read planes cost in expected squared score error
+    (section 方法二: reading a plane divides the channel's error variance by 4,
+    and the error enters every head's score through q_{g,j}).
+
+    Keys k_ij = sigma_j z_i share one standard-normal column z and the
+    sigma_j are powers of two, so every channel has the same codes and block
+    scales up to its power of two: the squared score error of channel j read
+    alone at depth t, measured against the full-precision keys through
+    orc_pack and orc_scan, is exactly sigma_j^2 sum_g q_{g,j}^2 MSE_z(t).
+    Its ratio to orc_importance must therefore be one constant over the
+    channels at every depth; sigma in place of sigma^2, or (sum_g q)^2 in
+    place of sum_g q^2, breaks that.  From depth 2 on each further plane
+    divides the error by about 4."""
+    rng = np.random.default_rng(11)
+    D, G, n, n_cal = 8, 4, 64 * 256, 4096
+    sig = 2.0 ** np.array([-2, -1, 0, 1, 2, 3, -3, 1], dtype=np.float64)
+    z = rng.standard_normal(n).astype(np.float32)
+    keys = (z[:, None].astype(np.float64) * sig[None, :]).astype(np.float32)[None]
+    q = rng.standard_normal((1, G, D)).astype(np.float32)
+    q[0, 1] = -0.5 * q[0, 0]        # mixed signs: sum_g q^2 and (sum_g q)^2 disagree
+    s2 = keys[:, :n_cal].astype(np.float64).var(axis=1).astype(np.float32)
+    w = orc.importance(s2, q)[0].astype(np.float64)
+    planes, scales = orc.pack(keys)
+    exact = q[0].astype(np.float64)[:, None, :] * keys[0].astype(np.float64)[None, :, :]   # [G][n][D]
+    err = {}
+    for t in (0, 1, 2, 3, 4):
+        e = np.zeros(D)
+        for j in range(D):
+            depth = np.zeros((1, D), np.uint8)
+            depth[0, j] = t
+            sc = orc.scan(planes, scales, depth, q, n, with_l1=False)[0]   # [G][n]
+            e[j] = np.mean(np.sum((exact[:, :, j] - sc) ** 2, axis=0))
+        ratio = e / w
+        assert np.allclose(ratio, ratio[0], rtol=1e-5), (t, ratio)
+        err[t] = e
+        for alt in (np.sqrt(s2[0]) * np.sum(q[0].astype(np.float64) ** 2, axis=0),
+                    s2[0] * np.sum(q[0].astype(np.float64), axis=0) ** 2):
+            r = e / alt
+            assert not np.allclose(r, r[0], rtol=1e-2)
+    for t in (2, 3):
+        assert np.all((err[t] / err[t + 1] > 3.0) & (err[t] / err[t + 1] < 6.0)), err[t] / err[t + 1]
+
+
 def plan_from_w(orc, w, B):
     """Plan with G = 1, q = 1 so that the importance is exactly w."""
     w = np.asarray(w, np.float32)
