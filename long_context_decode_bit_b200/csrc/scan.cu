@@ -495,14 +495,22 @@ scan_kernel(const ScanArgs a)
                     }
                 };
                 // Survivor mask over (head, token): one compare per score and
-                // no branch; then one pass per survivor, usually none.
+                // no branch; then one pass per survivor, usually none.  A NaN
+                // score counts as reaching tau, as it ranks above every number
+                // in the top-k's order (a head of NaN scores then overflows and
+                // is rerun densely).  Without a threshold sample every key is
+                // kept, so that each key's own slot is written.
                 using Mask = typename std::conditional<(G <= 4), uint32_t, unsigned long long>::type;
                 Mask mask = 0;
+                if (S.direct[0]) {   // the same for every head of a launch: n alone decides it
+                    mask = static_cast<Mask>(~static_cast<Mask>(0) >> (8 * sizeof(Mask) - 8 * G));
+                } else {
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float tau = S.tau[g];
+                    for (int g = 0; g < G; ++g) {
+                        const float tau = S.tau[g];
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) mask |= static_cast<Mask>(acc_at<G>(acc, m, g) >= tau) << (g * 8 + m);
+                        for (int m = 0; m < 8; ++m) mask |= static_cast<Mask>(!(acc_at<G>(acc, m, g) < tau)) << (g * 8 + m);
+                    }
                 }
                 while (mask) {
                     const int bit = (G <= 4 ? __ffs(static_cast<uint32_t>(mask)) : __ffsll(static_cast<long long>(mask))) - 1;

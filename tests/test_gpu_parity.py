@@ -191,6 +191,41 @@ def test_candidate_path_equals_dense(fathom_gpu, orc, budget):
     assert fathom_gpu.device_status() == fathom_gpu.OK
 
 
+@pytest.mark.parametrize("n", [2000, 20000], ids=["direct", "sampled"])
+def test_nan_query_channel_candidate_equals_dense(fathom_gpu, orc, n):
+    """A non-finite query channel (device memory: no host check sees it)
+    makes one head's scores NaN.  NaN ranks above every number in the
+    top-k's order, so the candidate path must keep such keys: without a
+    threshold sample every key sits at its own slot, and with one a NaN
+    score counts as reaching tau (a head of NaN scores then overflows and is
+    the dense rerun's business).  Every group the candidate path proves
+    exact equals the dense path's top-k and union."""
+    w = dataclasses.replace(inputs.TINY, name=f"nan-{n}", H=2, n=n, k=64, seed=91)
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    depth = np.zeros((w.H, w.D), np.uint8)
+    depth[:, :40] = 1
+    depth[:, 5] = 3
+    act, na = depth_to_active(depth)
+    active = torch.from_numpy(act.view(np.int16)).to(DEV)
+    n_active = torch.from_numpy(na).to(DEV)
+    q[0, 1, 5] = float("nan")
+    dense = fathom_gpu.scan(planes, scales, w.n, active, n_active, q)
+    d_idx, d_uni, d_cnt = fathom_gpu.topk(w.H, w.G, w.n, w.k, scores=dense)
+    cand = fathom_gpu.scan(planes, scales, w.n, active, n_active, q, fathom_gpu.SCAN_CANDIDATE, w.k)
+    c_idx, c_uni, c_cnt = fathom_gpu.topk(w.H, w.G, w.n, w.k, cand=cand)
+    torch.cuda.synchronize()
+    assert torch.isnan(dense[0, 1]).all() and not torch.isnan(dense[0, 0]).any() and not torch.isnan(dense[1]).any()
+    assert np.array_equal(d_idx[0, 1].cpu().numpy(), np.arange(w.k))   # equal NaN keys: lowest indices
+    proved = (c_cnt >= 0).cpu().numpy()
+    assert proved[1]
+    if n <= 2048:   # one scan tile: no threshold sample
+        assert proved.all()
+    for h in range(w.H):
+        if proved[h]:
+            assert torch.equal(c_idx[h], d_idx[h]) and torch.equal(c_uni[h], d_uni[h]) and c_cnt[h] == d_cnt[h]
+
+
 def test_candidate_overflow_is_flagged_and_repaired(fathom_gpu, orc):
     # Budget 0: every score is 0, so every key reaches the sampled threshold
     # and the candidate buffer overflows; the group must be flagged, and the
