@@ -18,9 +18,16 @@
 // cudaGetSymbolAddress (with that device current) and caches it.
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace fathom {
+
+// Defined in api.cu.
+int topk_cand_args_check(int G, int64_t n, int k, const int32_t* idx, const int32_t* union_idx,
+                         const int32_t* union_count);
+
 namespace {
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[FATHOM_NOALLOC_SCRATCH_BYTES];
@@ -59,16 +66,22 @@ extern "C" int fathom_scan_topk_noalloc(const uint64_t* planes, const uint16_t* 
     if (H < 0 || n < 0 || G < 1 || G > kMaxG) return H < 0 || n < 0 ? FATHOM_ERR_INVALID_ARG : FATHOM_ERR_UNSUPPORTED;
     if (H == 0) return FATHOM_OK;
     if (k < 1 || k > n) return FATHOM_ERR_INVALID_ARG;
+    // The top-k outputs are checked before the scan enqueues anything.
+    int st = topk_cand_args_check(G, n, k, idx, union_idx, union_count);
+    if (st != FATHOM_OK) return st;
     const size_t need = fathom_scan_cand_bytes(H, G, n, k);
     if (need == 0) return FATHOM_ERR_INVALID_ARG;
     if (need > FATHOM_NOALLOC_SCRATCH_BYTES) return FATHOM_ERR_WORKSPACE;
     void* scratch = nullptr;
-    const int st = scratch_for_current_device(&scratch);
+    st = scratch_for_current_device(&scratch);
     if (st != FATHOM_OK) return st;
+    nvtxRangePushA("fathom_scan_topk_noalloc");
     // The threshold pass resets the counters it needs, so the array's
     // leftover contents from an earlier call do not matter.
-    const int s1 = fathom_scan(planes, scales, H, D, n, nb_stride, active, n_active, q, G, FATHOM_SCAN_CANDIDATE,
-                               nullptr, scratch, need, k, stream);
-    if (s1 != FATHOM_OK) return s1;
-    return fathom_topk(nullptr, scratch, H, G, n, k, idx, union_idx, union_count, nullptr, 0, stream);
+    st = fathom_scan(planes, scales, H, D, n, nb_stride, active, n_active, q, G, FATHOM_SCAN_CANDIDATE, nullptr,
+                     scratch, need, k, stream);
+    if (st == FATHOM_OK)
+        st = fathom_topk(nullptr, scratch, H, G, n, k, idx, union_idx, union_count, nullptr, 0, stream);
+    nvtxRangePop();
+    return st;
 }

@@ -8,6 +8,7 @@ Its results must equal those of the allocating path, fathom_scan in
 CANDIDATE mode followed by fathom_topk, on two calls in a row (the second
 call reuses the array the first one left behind).  This file is collected
 last so a stop-at-first-failure run has already run every other test."""
+import ctypes
 import dataclasses
 
 import pytest
@@ -62,3 +63,29 @@ def test_noalloc_rejects_sizes_beyond_its_array(fathom_gpu):
                                       fathom._p(active), fathom._p(na), fathom._p(q), w.G, w.k, fathom._p(idx),
                                       fathom._p(uni), fathom._p(cnt), fathom._stream(None))
     assert st == fathom.ERR_WORKSPACE
+
+
+def test_noalloc_takes_no_device_memory_and_checks_outputs_first(fathom_gpu):
+    """A call after the first on a device takes no device memory: the free
+    memory the driver reports is the same before and after it.  Bad output
+    pointers are rejected before any work is enqueued."""
+    fathom = fathom_gpu
+    w = dataclasses.replace(inputs.LAYER_32K, name="noalloc-mem", H=4)
+    planes, scales, active, na, q = _setup(fathom, w, 48)
+    out = (torch.empty((w.H, w.G, w.k), dtype=torch.int32, device="cuda"),
+           torch.empty((w.H, w.G * w.k), dtype=torch.int32, device="cuda"),
+           torch.empty(w.H, dtype=torch.int32, device="cuda"))
+    fathom.scan_topk_noalloc(planes, scales, w.n, active, na, q, w.k, out=out)   # first call: one-time set-up
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    fathom.scan_topk_noalloc(planes, scales, w.n, active, na, q, w.k, out=out)
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    assert free0 == free1
+    assert torch.all(out[2] >= 0)
+    lib = fathom.lib()
+    misaligned = ctypes.c_void_p(out[0].data_ptr() + 2)
+    st = lib.fathom_scan_topk_noalloc(fathom._p(planes), fathom._p(scales), w.H, w.D, w.n, planes.shape[-1],
+                                      fathom._p(active), fathom._p(na), fathom._p(q), w.G, w.k, misaligned,
+                                      fathom._p(out[1]), fathom._p(out[2]), fathom._stream(None))
+    assert st == fathom.ERR_UNSUPPORTED
