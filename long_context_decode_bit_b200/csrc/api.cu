@@ -1,6 +1,12 @@
 // extern "C" entry points of libfathom.so (declared in include/fathom.h):
-// argument validation on the host, then the launches.  No allocation, no
-// state beyond the per-thread last CUDA error.
+// argument validation on the host, then the launches.  No allocation.  The
+// library's state is the per-thread last CUDA error code, one fault word per
+// device (fault.cu) and the scratch array of the allocation-free entry point
+// (noalloc.cu).  Every entry point that enqueues work opens an NVTX range
+// named after it, so that a trace shows the library's calls on the host
+// timeline (a no-op unless a profiler is attached).
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace fathom {
@@ -35,6 +41,14 @@ int launch_union_attention(const void* k, const void* v, int kv_dtype, int64_t H
                            float scale, float* out, void* ws, cudaStream_t stream);
 
 static thread_local int g_last_cuda_error = 0;
+
+// NVTX range over one library call.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int cuda_status(cudaError_t e)
 {
@@ -136,6 +150,23 @@ __global__ void nibbles_kernel(const uint64_t* __restrict__ planes, int64_t rows
 
 
 }  // namespace
+
+// Checks of fathom_topk's output arguments and limits for the candidate
+// path, shared with fathom_scan_topk_noalloc so that it rejects bad outputs
+// before it enqueues anything.
+int topk_cand_args_check(int G, int64_t n, int k, const int32_t* idx, const int32_t* union_idx,
+                         const int32_t* union_count)
+{
+    if (G < 1 || G > kMaxG) return FATHOM_ERR_UNSUPPORTED;
+    if (k < 1 || k > n) return FATHOM_ERR_INVALID_ARG;
+    if (k > kMaxK || k > kMaxCandK || static_cast<int64_t>(G) * k > kMaxUnion) return FATHOM_ERR_UNSUPPORTED;
+    if (!aligned(idx, 4) || !aligned(union_idx, 4) || !aligned(union_count, 4)) return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY_IN(check_device_ptr(idx));
+    FATHOM_TRY_IN(check_device_ptr(union_idx));
+    FATHOM_TRY_IN(check_device_ptr(union_count));
+    return FATHOM_OK;
+}
+
 }  // namespace fathom
 
 using namespace fathom;
@@ -176,6 +207,7 @@ int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, in
                 int64_t key_stride_tok, uint64_t* planes, uint16_t* scales, int64_t nb_stride,
                 fathom_stream_t stream)
 {
+    NvtxRange range("fathom_pack");
     if (H < 0 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
     if (key_dtype != FATHOM_KEYS_F32 && key_dtype != FATHOM_KEYS_BF16) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
@@ -203,6 +235,7 @@ int fathom_layer_budgets(const float* sigma2, const float* q, int64_t H, int G, 
                          int64_t total_bits, int32_t* budget_bits, void* workspace, size_t ws_bytes,
                          fathom_stream_t stream)
 {
+    NvtxRange range("fathom_layer_budgets");
     if (H < 0 || H > 0x7FFFFFFF || layers < 1 || layers > 1024 || total_bits < 0) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
     if (H == 0) return FATHOM_OK;
@@ -228,6 +261,7 @@ int fathom_calibrate(const void* keys, int key_dtype, int64_t H, int64_t n, int 
                      int64_t key_stride_tok, float* mean, float* sigma2, float* cov, void* workspace, size_t ws_bytes,
                      fathom_stream_t stream)
 {
+    NvtxRange range("fathom_calibrate");
     if (H < 0 || n < 0 || n >= (1LL << 40)) return FATHOM_ERR_INVALID_ARG;
     if (key_dtype != FATHOM_KEYS_F32 && key_dtype != FATHOM_KEYS_BF16) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
@@ -259,6 +293,7 @@ int fathom_union_attention(const void* k_cache, const void* v_cache, int kv_dtyp
                            const int32_t* union_count, int64_t M, float scale, float* out, void* workspace,
                            size_t ws_bytes, fathom_stream_t stream)
 {
+    NvtxRange range("fathom_union_attention");
     if (H < 0 || n < 0 || n >= (1LL << 31) || M < 1 || M > 65536) return FATHOM_ERR_INVALID_ARG;
     if (kv_dtype != FATHOM_KEYS_F32 && kv_dtype != FATHOM_KEYS_BF16) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
@@ -286,6 +321,7 @@ int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D, co
                 int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
                 fathom_stream_t stream)
 {
+    NvtxRange range("fathom_plan");
     if (H < 0 || H > 0x7FFFFFFF) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
     if (!budget_bits && (budget_flat < 0 || budget_flat > 4 * D)) return FATHOM_ERR_INVALID_ARG;
@@ -307,6 +343,7 @@ int fathom_plan(const float* sigma2, const float* q, int64_t H, int G, int D, co
 int fathom_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits, uint8_t* depth, uint16_t* active,
                       int32_t* n_active, fathom_stream_t stream)
 {
+    NvtxRange range("fathom_plan_fixed");
     if (H < 0 || H > 0x7FFFFFFF) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
     if (r < 0 || r > D || bits < 1 || bits > kPlanes) return FATHOM_ERR_INVALID_ARG;
@@ -329,6 +366,7 @@ int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
                 const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
                 void* cand, size_t cand_bytes, int k, fathom_stream_t stream)
 {
+    NvtxRange range("fathom_scan");
     return fathom::scan_entry(planes, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, cand_bytes, k,
                       false, stream);
 }
@@ -337,6 +375,7 @@ int fathom_scan_nibbles(const uint64_t* nibbles, const uint16_t* scales, int64_t
                         int64_t nb_stride, const uint16_t* active, const int32_t* n_active, const float* q, int G,
                         int mode, float* scores, void* cand, size_t cand_bytes, int k, fathom_stream_t stream)
 {
+    NvtxRange range("fathom_scan_nibbles");
     return fathom::scan_entry(nibbles, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, cand_bytes, k,
                       true, stream);
 }
@@ -344,6 +383,7 @@ int fathom_scan_nibbles(const uint64_t* nibbles, const uint16_t* scales, int64_t
 int fathom_nibbles_from_planes(const uint64_t* planes, int64_t H, int D, int64_t n, int64_t nb_stride,
                                uint64_t* nibbles, fathom_stream_t stream)
 {
+    NvtxRange range("fathom_nibbles_from_planes");
     if (H < 0 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
     if (H == 0 || n == 0) return FATHOM_OK;
@@ -368,6 +408,7 @@ int fathom_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
                 int32_t* union_idx, int32_t* union_count, void* workspace, size_t ws_bytes,
                 fathom_stream_t stream)
 {
+    NvtxRange range("fathom_topk");
     (void)workspace; (void)ws_bytes;
     if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
     if (G < 1 || G > kMaxG) return FATHOM_ERR_UNSUPPORTED;
@@ -395,6 +436,7 @@ int fathom_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t 
                         int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count, int bits,
                         float* out, fathom_stream_t stream)
 {
+    NvtxRange range("fathom_dequant_rows");
     if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31) || M < 0 || M > (1LL << 24)) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
     if (bits < 1 || bits > kPlanes) return FATHOM_ERR_INVALID_ARG;
