@@ -17,7 +17,8 @@ from _util import SCORE_RTOL, assert_topk_sets_match, keys_for_oracle, np_u16, n
 
 pytestmark = pytest.mark.gpu
 
-SAMPLED_GROUPS = (0, 157)   # first group, and one from the middle layers
+# 16 groups spread over all 36 layers of the step (first and last included)
+SAMPLED_GROUPS = tuple(int(h) for h in np.linspace(0, 287, 16).round())
 
 
 @pytest.fixture(scope="module")
@@ -94,7 +95,7 @@ def test_step_128k_sampled_groups(orc):
     torch.cuda.synchronize()
     d_ref = orc.plan(s2.cpu().numpy(), q.cpu().numpy(), 48)[0]
     assert np.array_equal(st.plan_out[0].cpu().numpy(), d_ref)
-    for h in (5, 287):
+    for h in (int(x) for x in np.linspace(5, 287, 16).round()):
         k = inputs.keys(w, h, h + 1, device="cuda")
         p_ref, s_ref = orc.pack(keys_for_oracle(k), nb_stride=planes.shape[-1])
         assert np.array_equal(np_u64(planes[h:h + 1]), p_ref)
@@ -102,3 +103,4 @@ def test_step_128k_sampled_groups(orc):
         ref, l1 = orc.scan(p_ref, s_ref, d_ref[h:h + 1], qn, w.n)
         r_idx = orc.topk(ref, w.k)[0]
         assert_topk_sets_match(idx[h:h + 1].cpu().numpy(), r_idx, ref, l1, w.k)
+        assert int(cnt[h]) > 0
