@@ -40,6 +40,7 @@
 // strided subset of tiles to the candidate buffer's sample area; CANDIDATE
 // keeps keys whose score reaches the head's threshold: at their own index
 // when there is no threshold sample, else in this tile's slot range.
+#include <cstdlib>
 #include <type_traits>
 
 #include "common.cuh"
@@ -91,6 +92,9 @@ struct ScanArgs {
     int mode;
     int32_t* fault;            // device fault word: set when a ring wait ran out
     bool nib;                  // `planes` is the nibble store, read at 4 bits
+#ifdef FATHOM_TEST_HOOKS
+    bool withhold;             // test build: withhold one ring arrival (see the producer)
+#endif
 };
 
 // Heads are handled in pairs for the packed FMA; odd G gets a zero pad.
@@ -405,6 +409,14 @@ scan_kernel(const ScanArgs a)
                 const uint16_t* src = a.scales + (h * D + j) * a.nb_stride + (bytes ? b0 + 8 * part : 0);
                 cp_async16(&S.rawscale[st][c * kScanTileBlocks + 8 * part], src, bytes);
             }
+#ifdef FATHOM_TEST_HOOKS
+            // Test build only: lane 0 of the first CTA of head 0 withholds its
+            // arrival for the first unit, so that stage never fills, every
+            // consumer wait on it runs out, and then this warp's wait for the
+            // stage to be freed runs out too.  Its copies still land (the
+            // next arrival and the final wait cover them).
+            if (a.withhold && u == 0 && lane == 0 && blockIdx.x == 0 && h == 0) continue;
+#endif
             cp_async_arrive(full0 + 8 * st);   // this lane's share of unit u
         }
         cp_async_wait_all();
@@ -635,6 +647,12 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
 {
     ScanArgs a{};
     a.nib = nib;
+#ifdef FATHOM_TEST_HOOKS
+    {
+        const char* e = getenv("FATHOM_TEST_WITHHOLD_ARRIVAL");
+        a.withhold = e != nullptr && e[0] == '1';
+    }
+#endif
     {
         const int st = device_fault_word(&a.fault);
         if (st) return st;
