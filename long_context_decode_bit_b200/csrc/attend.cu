@@ -191,11 +191,10 @@ int launch_attend_g(AttArgs a, int64_t H, cudaStream_t stream)
 {
     const int slices = kAttThreads / a.D;
     const size_t smem = sizeof(float) * (G * a.D + G * kAttRows + slices * G * a.D) + sizeof(int) * kAttRows;
-    cudaError_t e = cudaFuncSetAttribute(attend_chunk_kernel<DT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_status(e);
+    int st = ensure_dynamic_smem(reinterpret_cast<const void*>(attend_chunk_kernel<DT, G>), smem);
+    if (st) return st;
     attend_chunk_kernel<DT, G><<<dim3(a.chunks, static_cast<unsigned>(H)), kAttThreads, smem, stream>>>(a);
-    const int st = launch_status();
+    st = launch_status();
     if (st) return st;
     attend_combine_kernel<G><<<static_cast<unsigned>(H), kAttThreads, 0, stream>>>(a);
     return launch_status();

@@ -189,9 +189,8 @@ int launch_calibrate_t(const void* keys, int64_t H, int64_t n, int D, int64_t sh
         if (status) return status;
         if (cov) {
             const size_t smem = sizeof(double) * (kCovTile + 1) * D;
-            e = cudaFuncSetAttribute(calib_cov_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem));
-            if (e != cudaSuccess) return cuda_status(e);
+            status = ensure_dynamic_smem(reinterpret_cast<const void*>(calib_cov_kernel<DT>), smem);
+            if (status) return status;
             const int nbk = D / 8;
             const dim3 gc(static_cast<unsigned>(ceil_div(n, kCovChunk)), static_cast<unsigned>(H),
                           static_cast<unsigned>(ceil_div(static_cast<int64_t>(nbk) * nbk, kCalThreads)));

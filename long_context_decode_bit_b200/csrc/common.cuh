@@ -29,6 +29,40 @@ inline int launch_status() { return cuda_status(cudaGetLastError()); }
 // wait gave up; see fault.cu).
 int device_fault_word(int32_t** out);
 
+// Programmatic dependent launch for the kernels of a decode step (plan,
+// scans, threshold, top-k, union): each is launched so that the next one's
+// CTAs can become resident while it finishes.  A kernel calls pdl_wait()
+// before it reads anything an earlier kernel wrote, and lets its successor
+// launch (pdl_launch_dependents) only after that wait; so when any kernel's
+// wait returns, every kernel before it in the stream has completed and its
+// writes are visible.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...));
+}
+
+// SM count of the current device (queried once per device; launch.cu).
+int device_sm_count(int* sms);
+
+// Raise `func`'s dynamic shared memory limit on the current device to at
+// least `bytes`; the driver is called only the first time (or for a larger
+// size).  launch.cu.
+int ensure_dynamic_smem(const void* func, size_t bytes);
+
 // ---------------------------------------------------------------------
 // Order-preserving map from fp32 to uint32: larger float -> larger key.
 // -0 is folded onto +0 so that the two compare equal, as fp32 values do.

@@ -4,11 +4,13 @@
 // channel j is worth the item w_j * 4^-t; the water level theta* is the
 // smallest theta whose item count above it fits the budget, and each
 // channel's depth is its number of items above theta*.  One CTA plans one
-// group, one thread per channel.  theta is searched by bisection over an
-// integer key that orders items exactly and grows like log2(theta): the
-// fp32 exponent and fraction of w, with the exponent extended below the
-// subnormal range and lowered by 2t for the factor 4^-t.
+// group, one thread per channel.  Items are compared through an integer key
+// that orders them exactly and grows like log2 of the item: the fp32
+// exponent and fraction of w, with the exponent extended below the
+// subnormal range and lowered by 2t for the factor 4^-t.  The level is the
+// (B+1)-th largest item key, found by a radix select over the 4 D keys.
 #include "common.cuh"
+#include "select.cuh"
 
 namespace fathom {
 
@@ -63,10 +65,11 @@ __global__ void plan_kernel(const float* __restrict__ sigma2, const float* __res
                             int32_t* __restrict__ n_active, float* __restrict__ theta)
 {
     __shared__ int warp_cnt[kMaxD / 32];
-    __shared__ int red_min[kMaxD / 32], red_max[kMaxD / 32];
+    __shared__ int32_t key0[kMaxD];
     const int64_t h = blockIdx.x;
     const int j = threadIdx.x;   // blockDim.x == D
-    const int lane = j & 31, warp = j >> 5, nwarps = D >> 5;
+    pdl_wait();
+    pdl_launch_dependents();
 
     // Importance in the plan's fixed single-precision order (no FMA).
     const float* qh = q + h * G * D + j;
@@ -78,8 +81,7 @@ __global__ void plan_kernel(const float* __restrict__ sigma2, const float* __res
     int B = budget_bits ? budget_bits[h] : budget_flat;
     B = min(max(B, 0), 4 * D);
 
-    int32_t k0 = 0, k3 = 0;
-    if (pos) { k0 = item_key(w, 0); k3 = item_key(w, 3); }
+    const int32_t k0 = pos ? item_key(w, 0) : 0;
     const int npos = __syncthreads_count(pos);
 
     int32_t kstar;          // items with key > kstar are read
@@ -88,27 +90,23 @@ __global__ void plan_kernel(const float* __restrict__ sigma2, const float* __res
         all_positive = true;
         kstar = 0;
     } else {
-        // Range of item keys, for the bisection bounds.
-        int32_t mn = pos ? k3 : INT32_MAX, mx = pos ? k0 : INT32_MIN;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        if (lane == 0) { red_min[warp] = mn; red_max[warp] = mx; }
+        // kstar is the (B+1)-th largest item key: the smallest level with at
+        // most B items above it.  Item t of channel j has the key
+        // k0_j - t * 2^24 (the exponent lowered by 2t); a block radix select
+        // over the 4 D items finds it in three passes.  Channels that read
+        // nothing give the key 0, below every real item, and as 4 npos > B
+        // they never reach rank B + 1.
+        __shared__ uint32_t hist[kRadixBins];
+        __shared__ uint32_t sh[2];
+        key0[j] = pos ? k0 : INT32_MIN;   // INT32_MIN: no items (every real key is far above it)
         __syncthreads();
-        mn = INT32_MAX; mx = INT32_MIN;
-        for (int wi = 0; wi < nwarps; ++wi) { mn = min(mn, red_min[wi]); mx = max(mx, red_max[wi]); }
-        // Invariant: count(lo) > B >= count(hi); count(K) = #items with key > K.
-        int64_t lo = static_cast<int64_t>(mn) - 1, hi = mx;
-        int32_t kj[4] = {k0, pos ? item_key(w, 1) : 0, pos ? item_key(w, 2) : 0, k3};
-        while (hi - lo > 1) {
-            const int64_t mid = lo + ((hi - lo) >> 1);
-            int c = 0;
-            for (int r = 0; r < 4; ++r) c += __syncthreads_count(pos && kj[r] > mid);
-            if (c <= B) hi = mid; else lo = mid;
-        }
-        kstar = static_cast<int32_t>(hi);
+        auto key_at = [&](int64_t i) -> uint32_t {
+            const int32_t c = key0[i >> 2];
+            if (c == INT32_MIN) return 0u;
+            return static_cast<uint32_t>(c - static_cast<int32_t>(i & 3) * (1 << 24)) ^ 0x80000000u;
+        };
+        const Select r = block_select(key_at, 4LL * D, B + 1, hist, sh);
+        kstar = static_cast<int32_t>(r.T ^ 0x80000000u);
     }
 
     int t = 0;
@@ -261,9 +259,8 @@ int launch_plan(const float* sigma2, const float* q, int64_t H, int G, int D, co
                 int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
                 cudaStream_t stream)
 {
-    plan_kernel<<<static_cast<unsigned>(H), D, 0, stream>>>(sigma2, q, G, D, budget_bits, budget_flat,
-                                                          depth, active, n_active, theta);
-    return launch_status();
+    return launch_pdl(plan_kernel, dim3(static_cast<unsigned>(H)), dim3(D), 0, stream, sigma2, q, G, D, budget_bits,
+                      budget_flat, depth, active, n_active, theta);
 }
 
 int launch_plan_fixed(const float* q, int64_t H, int G, int D, int r, int bits, uint8_t* depth, uint16_t* active,

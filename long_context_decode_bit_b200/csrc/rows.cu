@@ -70,9 +70,8 @@ int launch_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t 
                         float* out, cudaStream_t stream)
 {
     const size_t smem = sizeof(float) * kRowsPerCta * (D + 1);
-    const cudaError_t e = cudaFuncSetAttribute(dequant_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_status(e);
+    const int st = ensure_dynamic_smem(reinterpret_cast<const void*>(dequant_rows_kernel), smem);
+    if (st) return st;
     const dim3 grid(static_cast<unsigned>(ceil_div(M, kRowsPerCta)), static_cast<unsigned>(H));
     dequant_rows_kernel<<<grid, kRowsThreads, smem, stream>>>(planes, scales, D, n, nb_stride, rows, M, row_count,
                                                               bits, out);

@@ -278,6 +278,8 @@ scan_kernel(const ScanArgs a)
     const int64_t h = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int D = a.D;
+    pdl_wait();
+    pdl_launch_dependents();
     const int na = min(max(a.n_active[h], 0), D);   // trust nothing beyond D entries
 
     // ---- the group's plan: one parallel read of the active list, then a
@@ -556,24 +558,23 @@ template <int G, bool NIB>
 int launch_scan_g(ScanArgs a, int64_t ltiles, unsigned H, cudaStream_t stream)
 {
     const size_t smem = sizeof(SharedScan<G>);
-    const cudaError_t e = cudaFuncSetAttribute(scan_kernel<G, NIB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_status(e);
+    int st = ensure_dynamic_smem(reinterpret_cast<const void*>(scan_kernel<G, NIB>), smem);
+    if (st) return st;
     // Several tiles per CTA amortise the per-CTA plan set-up: as many as
     // keep the grid at two or more waves of resident CTAs (capped).
 #ifndef FATHOM_SCAN_WAVES
 #define FATHOM_SCAN_WAVES 2
 #endif
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int sms = 0;
+    st = device_sm_count(&sms);
+    if (st) return st;
     const int64_t slots = static_cast<int64_t>(sms) * scan_min_ctas<G>() * FATHOM_SCAN_WAVES;
     int64_t per = ceil_div(ltiles * static_cast<int64_t>(H), slots);
     per = per < 1 ? 1 : (per > FATHOM_SCAN_TILES_CAP ? FATHOM_SCAN_TILES_CAP : per);
     per = ceil_div(ltiles, ceil_div(ltiles, per));   // the same CTAs per group, their tiles evened out
     a.tiles_per_cta = static_cast<int>(per);
     const unsigned gx = static_cast<unsigned>(ceil_div(ltiles, a.tiles_per_cta));
-    scan_kernel<G, NIB><<<dim3(gx, H), kScanThreads, smem, stream>>>(a);
-    return launch_status();
+    return launch_pdl(scan_kernel<G, NIB>, dim3(gx, H), dim3(kScanThreads), smem, stream, a);
 }
 
 template <bool NIB>

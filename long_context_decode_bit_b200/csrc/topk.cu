@@ -13,6 +13,7 @@
 // sort on 64-bit composite keys.  The same select, over per-thread maxima
 // of the sample scores, picks the candidate threshold tau.
 #include "common.cuh"
+#include "select.cuh"
 
 namespace fathom {
 
@@ -20,84 +21,7 @@ namespace {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkCandThreads = 512;   // candidate lists are short: smaller CTAs, more of them per SM
-constexpr int kRadixBins = 2048;
 constexpr int kMaxTies = 4096;
-constexpr unsigned kFull = 0xffffffffu;
-
-struct Select {
-    uint32_t T;     // k-th largest key
-    int take_eq;    // keys equal to T that belong to the top k (>= 1)
-};
-
-// k-th largest of key_at(0 .. count-1), 1 <= kk <= count.  All threads of the
-// CTA must call it.  hist: kRadixBins words of shared memory; sh: 2 ints.
-template <class KeyAt>
-__device__ Select block_select(KeyAt key_at, int64_t count, int kk, uint32_t* hist, uint32_t* sh)
-{
-    uint32_t prefix = 0, mask = 0;
-#pragma unroll
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int width = pass == 2 ? 10 : 11;
-        const uint32_t dmask = (1u << width) - 1u;
-        const int nbins = 1 << width;
-        for (int b = threadIdx.x; b < nbins; b += blockDim.x) hist[b] = 0;
-        __syncthreads();
-        for (int64_t i = threadIdx.x; i < count; i += blockDim.x) {
-            const uint32_t key = key_at(i);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            // Lane L owns bins [top - per, top), top = nbins - per*L: lane 0
-            // has the highest digits.  Find the digit holding the kk-th key.
-            const int lane = threadIdx.x, per = nbins / 32, top = nbins - per * lane;
-            uint32_t lsum = 0;
-            for (int b = top - 1; b >= top - per; --b) lsum += hist[b];
-            uint32_t incl = lsum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t v = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const uint32_t excl = incl - lsum;
-            const unsigned bal = __ballot_sync(kFull, excl < static_cast<uint32_t>(kk) &&
-                                                          static_cast<uint32_t>(kk) <= incl);
-            if (lane == __ffs(bal) - 1) {
-                uint32_t c = excl;
-                for (int b = top - 1; b >= top - per; --b) {
-                    if (c + hist[b] >= static_cast<uint32_t>(kk)) { sh[0] = b; sh[1] = c; break; }
-                    c += hist[b];
-                }
-            }
-        }
-        __syncthreads();
-        kk -= static_cast<int>(sh[1]);
-        prefix |= sh[0] << shift;
-        mask |= dmask << shift;
-        __syncthreads();
-    }
-    return Select{prefix, kk};
-}
-
-// In-place bitonic sort of n (a power of two) elements in shared memory.
-template <typename T, bool kDescending>
-__device__ void bitonic_sort(T* v, int n)
-{
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            __syncthreads();
-            for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
-                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
-                const bool up = (lo & size) == 0;
-                const T x = v[lo], y = v[hi];
-                const bool sw = kDescending ? (up ? (x < y) : (x > y)) : (up ? (x > y) : (x < y));
-                if (sw) { v[lo] = y; v[hi] = x; }
-            }
-        }
-    }
-    __syncthreads();
-}
 
 __device__ __forceinline__ uint64_t composite(uint32_t key, uint32_t idx)
 {
@@ -109,6 +33,14 @@ __host__ __device__ inline int pow2_at_least(int x)
     int p = 1;
     while (p < x) p <<= 1;
     return p;
+}
+
+// Sort buffer of a top-k CTA: the k winners' 64-bit composites, or up to
+// kMaxTies tie indices.
+__host__ __device__ inline size_t sort_tmp_bytes(int kpow2)
+{
+    const size_t a = sizeof(uint64_t) * kpow2, b = sizeof(int32_t) * kMaxTies;
+    return a > b ? a : b;
 }
 
 // Header of a group's candidate buffer: the threshold, and the counters reset.
@@ -138,11 +70,19 @@ tau_kernel(const float* __restrict__ sample, CandHeader* __restrict__ hdr, int64
     __shared__ uint32_t tmax[kTopkThreads];
     __shared__ uint32_t sh[2];
     const int64_t hg = blockIdx.x;
+    pdl_wait();
+    pdl_launch_dependents();
     float tau = -INFINITY;
     if (n_sample > 0) {
-        const float* s = sample + hg * n_sample;
+        // n_sample is a whole number of 2048-token tiles and the sample
+        // 16-byte aligned: float4 reads, several in flight per thread.
+        const float4* s4 = reinterpret_cast<const float4*>(sample + hg * n_sample);
         uint32_t mk = 0;   // order key of the thread's maximum (0: none, below every score's key)
-        for (int64_t i = threadIdx.x; i < n_sample; i += blockDim.x) mk = max(mk, order_key(s[i]));
+#pragma unroll 4
+        for (int64_t i = threadIdx.x; i < n_sample / 4; i += blockDim.x) {
+            const float4 x = s4[i];
+            mk = max(max(mk, order_key(x.x)), max(order_key(x.y), max(order_key(x.z), order_key(x.w))));
+        }
         tmax[threadIdx.x] = mk;
         __syncthreads();
         const Select r = block_select([&](int64_t i) { return tmax[i]; }, kTopkThreads, static_cast<int>(m_rank),
@@ -161,6 +101,8 @@ tau_kernel_large(const float* __restrict__ sample, CandHeader* __restrict__ hdr,
     __shared__ uint32_t hist[kRadixBins];
     __shared__ uint32_t sh[2];
     const int64_t hg = blockIdx.x;
+    pdl_wait();
+    pdl_launch_dependents();
     const float* s = sample + hg * n_sample;
     const Select r = block_select([&](int64_t i) { return order_key(s[i]); }, n_sample, static_cast<int>(m_rank),
                                   hist, sh);
@@ -169,31 +111,111 @@ tau_kernel_large(const float* __restrict__ sample, CandHeader* __restrict__ hdr,
 
 struct TopkArgs {
     const float* scores;        // dense [H*G][n] or null
-    const CandHeader* hdr;      // candidate mode
+    CandHeader* hdr;            // candidate mode (hdr[h*G].pad: the head's arrival counter)
     const int32_t* tile_counts; // [H*G][tiles] (with a threshold sample)
     const int2* entries;
     int64_t cap, tiles, tslot;
     int64_t n;
-    int k, kpow2;
+    int G, k, kpow2;
     int gather_cap;             // survivors gathered into shared memory (tile slots)
     int32_t* idx;               // [H*G][k]
+    int32_t* union_idx;         // [H][G*k]: group g's winners sorted by index at [g*k, g*k+k), then the union
+    int32_t* union_count;       // [H]
+    const int32_t* fault;       // device fault word
 };
 
-__global__ void __launch_bounds__(kTopkThreads)
-topk_kernel(const TopkArgs a)
+// Sorted, de-duplicated union of a group's G winner lists, each already
+// sorted by index, in shared memory (buf0[g*k .. g*k+k)).  The lists are
+// merged pairwise (ceil(log2 G) levels, between buf0 and buf1), equal
+// indices then sit side by side, and the first of each run is kept.
+// dst: the union, padded with -1 to G*k.  Every thread of the CTA must call
+// it; buf0 and buf1 hold G*k ints each.
+__device__ void merge_union(int32_t* buf0, int32_t* buf1, int G, int k, int32_t* dst, int32_t* union_count_h,
+                            int* warp_tot)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
+    const int gk = G * k;
+    int32_t* src = buf0;
+    int32_t* tmp = buf1;
+    for (int L = k; L < gk; L *= 2) {
+        merge_level<int32_t, false>(src, tmp, gk, L);
+        __syncthreads();
+        int32_t* t = src; src = tmp; tmp = t;
+    }
+    const int32_t* merged = src;
+    // Each thread owns a contiguous run of the merged order; keep first occurrences.
+    const int per = (gk + nt - 1) / nt;
+    const int lo = min(tid * per, gk), hi = min(lo + per, gk);
+    int mine = 0;
+    for (int i = lo; i < hi; ++i) mine += i == 0 || merged[i] != merged[i - 1];
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < (nt >> 5); ++w) {
+        const int v = warp_tot[w];
+        before += w < warp ? v : 0;
+        total += v;
+    }
+    int pos = before + incl - mine;
+    for (int i = lo; i < hi; ++i)
+        if (i == 0 || merged[i] != merged[i - 1]) dst[pos++] = merged[i];
+    for (int i = total + tid; i < gk; i += nt) dst[i] = -1;
+    if (tid == 0) *union_count_h = total;
+}
+
+// Load a head's G sorted lists from union_idx into shared memory (through L2:
+// other CTAs wrote them) and check them and the fault word; false if the
+// head must report a failure (written here).
+__device__ bool load_lists(const TopkArgs& a, int64_t h, int32_t* lists, int* failed)
+{
+    const int gk = a.G * a.k;
+    const int32_t* src = a.union_idx + h * gk;
+    if (threadIdx.x == 0) *failed = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < gk; i += blockDim.x) {
+        const int32_t x = __ldcg(src + i);
+        if (x < 0) *failed = 1;
+        lists[i] = x;
+    }
+    __syncthreads();
+    const int32_t faulted = __ldcg(a.fault);   // a scan whose ring wait gave up left void scores
+    if (*failed || faulted) {
+        for (int i = threadIdx.x; i < gk; i += blockDim.x) a.union_idx[h * gk + i] = -1;
+        if (threadIdx.x == 0) a.union_count[h] = faulted ? FATHOM_ERR_TIMEOUT : FATHOM_ERR_OVERFLOW;
+        return false;
+    }
+    return true;
+}
+
+// Per query head (h, g): the k winners, in (score desc, index asc) order to
+// idx, and sorted by index to the group's slice of union_idx.  A head that
+// cannot prove its top-k exact writes -1 to both.  Returns after its writes.
+__device__ void topk_head(const TopkArgs& a, unsigned char* smem)
+{
     uint64_t* win = reinterpret_cast<uint64_t*>(smem);                        // kpow2
     int32_t* ties = reinterpret_cast<int32_t*>(win + a.kpow2);               // kMaxTies
     uint32_t* hist = reinterpret_cast<uint32_t*>(ties + kMaxTies);           // kRadixBins
-    int2* gathered = reinterpret_cast<int2*>(hist + kRadixBins);             // gather_cap (tile slots)
+    unsigned char* tmp = reinterpret_cast<unsigned char*>(hist + kRadixBins);   // sort buffer (sort_tmp_bytes)
+    int2* gathered = reinterpret_cast<int2*>(tmp + sort_tmp_bytes(a.kpow2));     // gather_cap (tile slots)
     __shared__ uint32_t sh[2];
     __shared__ int w_cnt, t_cnt, warp_eq[kTopkThreads / 32], g_cnt, g_bad;
 
-    const int64_t hg = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+    const int g = blockIdx.x;
+    const int64_t h = blockIdx.y;
+    const int64_t hg = h * gridDim.x + g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.k;
     int32_t* out = a.idx + hg * k;
+    int32_t* sorted_out = a.union_idx + h * a.G * k + g * k;
+    auto fail = [&]() {
+        for (int r = tid; r < k; r += blockDim.x) { out[r] = -1; sorted_out[r] = -1; }
+    };
 
     int64_t count;
     const int2* ent = nullptr;
@@ -204,30 +226,46 @@ topk_kernel(const TopkArgs a)
     } else if (a.tslot == 0) {
         count = a.hdr[hg].count;            // every key kept at its own index
         ent = a.entries + hg * a.cap;
-        if (count < k || count > a.cap) {
-            for (int r = tid; r < k; r += blockDim.x) out[r] = -1;
-            return;
-        }
+        if (count < k || count > a.cap) { fail(); return; }
     } else {
-        // Gather the non-empty tile slots into shared memory.
+        // Gather the non-empty tile slots into shared memory: a warp scan of
+        // the tile counts gives each tile its place (one shared atomic per
+        // warp), and each thread copies its tile with several loads in flight.
         if (tid == 0) { g_cnt = 0; g_bad = 0; }
         __syncthreads();
         const int32_t* tc = a.tile_counts + hg * a.tiles;
         const int2* src = a.entries + hg * a.cap;
-        for (int64_t t = tid; t < a.tiles; t += blockDim.x) {
-            const int c = tc[t];
-            if (c <= 0) continue;
-            if (c > a.tslot) { g_bad = 1; continue; }       // slot overflowed: keys were dropped
-            const int base = atomicAdd(&g_cnt, c);
+        for (int64_t t0 = 0; t0 < a.tiles; t0 += blockDim.x) {
+            const int64_t t = t0 + tid;
+            int c = t < a.tiles ? tc[t] : 0;
+            if (c > a.tslot) { g_bad = 1; c = 0; }       // slot overflowed: keys were dropped
+            c = max(c, 0);
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int wbase = 0;
+            if (lane == 31 && incl > 0) wbase = atomicAdd(&g_cnt, incl);
+            wbase = __shfl_sync(kFull, wbase, 31);
+            const int base = wbase + incl - c;
+            if (c == 0) continue;
             if (base + c > a.gather_cap) { g_bad = 1; continue; }
-            for (int e = 0; e < c; ++e) gathered[base + e] = src[t * a.tslot + e];
+            const int2* sp = src + t * a.tslot;
+            for (int e0 = 0; e0 < c; e0 += 4) {
+                int2 x[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (e0 + u < c) x[u] = sp[e0 + u];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (e0 + u < c) gathered[base + e0 + u] = x[u];
+            }
         }
         __syncthreads();
         count = g_cnt;
-        if (g_bad || count < k || count > a.gather_cap) {   // could not prove exactness
-            for (int r = tid; r < k; r += blockDim.x) out[r] = -1;
-            return;
-        }
+        if (g_bad || count < k || count > a.gather_cap) { fail(); return; }   // could not prove exactness
         ent = gathered;
     }
     auto key_at = [&](int64_t i) -> uint32_t {
@@ -263,85 +301,91 @@ topk_kernel(const TopkArgs a)
             __syncthreads();
         }
     } else {
-        for (int64_t i = tid; i < count; i += blockDim.x) {
-            const uint32_t key = key_at(i);
-            if (key > sel.T) win[atomicAdd(&w_cnt, 1)] = composite(key, idx_at(i));
-            else if (key == sel.T) {
-                const int p = atomicAdd(&t_cnt, 1);
+        // Keys above T and ties at T, placed with one shared atomic per warp.
+        const unsigned below = (1u << lane) - 1u;
+        for (int64_t i0 = 0; i0 < count; i0 += blockDim.x) {
+            const int64_t i = i0 + tid;
+            uint32_t key = 0;
+            if (i < count) key = key_at(i);
+            const bool gt = i < count && key > sel.T;
+            const bool eq = i < count && key == sel.T;
+            const unsigned bg = __ballot_sync(kFull, gt), be = __ballot_sync(kFull, eq);
+            int wg = 0, we = 0;
+            if (lane == 0) {
+                if (bg) wg = atomicAdd(&w_cnt, __popc(bg));
+                if (be) we = atomicAdd(&t_cnt, __popc(be));
+            }
+            wg = __shfl_sync(kFull, wg, 0);
+            we = __shfl_sync(kFull, we, 0);
+            if (gt) win[wg + __popc(bg & below)] = composite(key, idx_at(i));
+            if (eq) {
+                const int p = we + __popc(be & below);
                 if (p < kMaxTies) ties[p] = static_cast<int32_t>(idx_at(i));
             }
         }
         __syncthreads();
-        if (t_cnt > kMaxTies) {
-            for (int r = tid; r < k; r += blockDim.x) out[r] = -1;
-            return;
-        }
+        if (t_cnt > kMaxTies) { fail(); return; }
         const int tp = pow2_at_least(t_cnt);
         for (int i = t_cnt + tid; i < tp; i += blockDim.x) ties[i] = INT32_MAX;
-        bitonic_sort<int32_t, false>(ties, tp);
+        block_sort<int32_t, false>(ties, reinterpret_cast<int32_t*>(tmp), tp);
         const int base = w_cnt;
         for (int r = tid; r < sel.take_eq; r += blockDim.x)
             win[base + r] = composite(sel.T, static_cast<uint32_t>(ties[r]));
     }
     __syncthreads();
     for (int i = k + tid; i < a.kpow2; i += blockDim.x) win[i] = 0;
-    bitonic_sort<uint64_t, true>(win, a.kpow2);
-    for (int r = tid; r < k; r += blockDim.x)
-        out[r] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(win[r] & 0xFFFFFFFFu));
+    block_sort<uint64_t, true>(win, reinterpret_cast<uint64_t*>(tmp), a.kpow2);
+    // Score order to idx; the same k indices sorted ascending to the group's
+    // slice of union_idx (ties[] is free again and holds kMaxTies >= kpow2).
+    for (int r = tid; r < a.kpow2; r += blockDim.x) {
+        const int32_t i = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(win[r] & 0xFFFFFFFFu));
+        if (r < k) out[r] = i;
+        ties[r] = r < k ? i : INT32_MAX;
+    }
+    block_sort<int32_t, false>(ties, reinterpret_cast<int32_t*>(tmp), a.kpow2);
+    for (int r = tid; r < k; r += blockDim.x) sorted_out[r] = ties[r];
 }
 
-// Sorted, de-duplicated union of a group's G winner lists.
 __global__ void __launch_bounds__(kTopkThreads)
-union_kernel(const int32_t* __restrict__ idx, int G, int k, int upow2, int32_t* __restrict__ union_idx,
-             int32_t* __restrict__ union_count, const int32_t* __restrict__ fault)
+topk_kernel(const TopkArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    int32_t* v = reinterpret_cast<int32_t*>(smem);
-    __shared__ int warp_tot[kTopkThreads / 32], failed;
+    pdl_wait();
+    pdl_launch_dependents();
+    topk_head(a, smem);
+    if (a.scores) return;   // dense: union_kernel follows
+    // Candidate mode: the last of a head's G CTAs to finish builds the head's
+    // union from the G sorted slices (fence, then one counter per head; the
+    // counter is reset by the threshold pass and again by the last CTA).
+    __shared__ int last, failed, warp_tot[kTopkThreads / 32];
+    const int64_t h = blockIdx.y;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&a.hdr[h * a.G].pad, 1) == a.G - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    if (threadIdx.x == 0) a.hdr[h * a.G].pad = 0;
+    // The head's own top-k is written: its shared memory is free for the union.
+    int32_t* lists = reinterpret_cast<int32_t*>(smem);
+    int32_t* merged = lists + a.G * a.k;
+    if (!load_lists(a, h, lists, &failed)) return;
+    merge_union(lists, merged, a.G, a.k, a.union_idx + h * a.G * a.k, a.union_count + h, warp_tot);
+}
+
+// The union after a dense top-k (one CTA per group).
+__global__ void __launch_bounds__(kTopkThreads)
+union_kernel(const TopkArgs a)
+{
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ int failed, warp_tot[kTopkThreads / 32];
     const int64_t h = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gk = G * k;
-    const int32_t* src = idx + h * gk;
-    int32_t* dst = union_idx + h * gk;
-    if (tid == 0) failed = 0;
-    __syncthreads();
-    for (int i = tid; i < upow2; i += blockDim.x) {
-        const int32_t x = i < gk ? src[i] : INT32_MAX;
-        if (x < 0) failed = 1;
-        v[i] = x;
-    }
-    __syncthreads();
-    const int32_t faulted = *fault;   // a scan whose ring wait gave up left void scores
-    if (failed || faulted) {
-        for (int i = tid; i < gk; i += blockDim.x) dst[i] = -1;
-        if (tid == 0) union_count[h] = faulted ? FATHOM_ERR_TIMEOUT : FATHOM_ERR_OVERFLOW;
-        return;
-    }
-    bitonic_sort<int32_t, false>(v, upow2);
-    // Each thread owns a contiguous run; keep first occurrences.
-    const int per = upow2 / blockDim.x > 0 ? upow2 / blockDim.x : 1;
-    const int lo = tid * per;
-    int mine = 0;
-    for (int i = lo; i < lo + per && i < upow2; ++i)
-        mine += (v[i] != INT32_MAX) && (i == 0 || v[i] != v[i - 1]);
-    int incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < (kTopkThreads / 32); ++w) {
-        if (w < warp) before += warp_tot[w];
-        total += warp_tot[w];
-    }
-    int pos = before + incl - mine;
-    for (int i = lo; i < lo + per && i < upow2; ++i)
-        if ((v[i] != INT32_MAX) && (i == 0 || v[i] != v[i - 1])) dst[pos++] = v[i];
-    for (int i = total + tid; i < gk; i += blockDim.x) dst[i] = -1;
-    if (tid == 0) union_count[h] = total;
+    pdl_wait();
+    pdl_launch_dependents();
+    int32_t* lists = reinterpret_cast<int32_t*>(smem);
+    int32_t* merged = lists + a.G * a.k;
+    if (!load_lists(a, h, lists, &failed)) return;
+    merge_union(lists, merged, a.G, a.k, a.union_idx + h * a.G * a.k, a.union_count + h, warp_tot);
 }
 
 }  // namespace
@@ -349,22 +393,23 @@ union_kernel(const int32_t* __restrict__ idx, int G, int k, int upow2, int32_t* 
 int launch_tau(const float* sample, CandHeader* hdr, int64_t heads, int64_t n_sample, int64_t m_rank,
                int64_t n_keys, cudaStream_t stream)
 {
+    const dim3 grid(static_cast<unsigned>(heads)), block(kTopkThreads);
     if (n_sample > 0 && m_rank * 8 > kTopkThreads)
-        tau_kernel_large<<<static_cast<unsigned>(heads), kTopkThreads, 0, stream>>>(sample, hdr, n_sample, m_rank,
-                                                                                  n_keys);
-    else
-        tau_kernel<<<static_cast<unsigned>(heads), kTopkThreads, 0, stream>>>(sample, hdr, n_sample, m_rank, n_keys);
-    return launch_status();
+        return launch_pdl(tau_kernel_large, grid, block, 0, stream, sample, hdr, n_sample, m_rank, n_keys);
+    return launch_pdl(tau_kernel, grid, block, 0, stream, sample, hdr, n_sample, m_rank, n_keys);
 }
 
 // Survivors one top-k CTA gathers: 8k, twice the ~4k a candidate pass keeps
 // (kCandGather at the largest k); more marks the group for the dense rerun.
 int gather_cap(int k) { return 8 * k < kCandGather ? 8 * k : kCandGather; }
 
-size_t topk_smem_bytes(int k, bool gather)
+size_t topk_smem_bytes(int G, int k, bool gather, bool fused_union)
 {
-    return sizeof(uint64_t) * pow2_at_least(k) + sizeof(int32_t) * kMaxTies + sizeof(uint32_t) * kRadixBins +
-           (gather ? sizeof(int2) * gather_cap(k) : 0);
+    const size_t own = sizeof(uint64_t) * pow2_at_least(k) + sizeof(int32_t) * kMaxTies +
+                       sizeof(uint32_t) * kRadixBins + sort_tmp_bytes(pow2_at_least(k)) +
+                       (gather ? sizeof(int2) * gather_cap(k) : 0);
+    const size_t uni = fused_union ? 2 * sizeof(int32_t) * G * k : 0;   // lists + merged order
+    return own > uni ? own : uni;
 }
 
 int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
@@ -373,15 +418,24 @@ int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
     TopkArgs a{};
     a.scores = scores;
     a.n = n;
+    a.G = G;
     a.k = k;
     a.kpow2 = pow2_at_least(k);
     a.gather_cap = gather_cap(k);
     a.idx = idx;
+    a.union_idx = union_idx;
+    a.union_count = union_count;
+    {
+        int32_t* fault = nullptr;
+        const int st = device_fault_word(&fault);
+        if (st) return st;
+        a.fault = fault;
+    }
     bool gather = false;
     if (!scores) {
         const CandLayout L = cand_layout(H, G, n, k);
-        const char* base = static_cast<const char*>(cand);
-        a.hdr = reinterpret_cast<const CandHeader*>(base + L.off_hdr);
+        char* base = static_cast<char*>(const_cast<void*>(cand));
+        a.hdr = reinterpret_cast<CandHeader*>(base + L.off_hdr);
         a.tile_counts = reinterpret_cast<const int32_t*>(base + L.off_counts);
         a.entries = reinterpret_cast<const int2*>(base + L.off_entries);
         a.cap = L.cap;
@@ -389,25 +443,19 @@ int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t
         a.tslot = L.tslot;
         gather = L.tslot > 0;
     }
-    const size_t smem = topk_smem_bytes(k, gather);
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_status(e);
+    const size_t smem = topk_smem_bytes(G, k, gather, scores == nullptr);
+    int st = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_kernel), smem);
+    if (st) return st;
     // The dense path's index-ordered pass counts per warp over kTopkThreads
-    // threads; candidate lists take smaller CTAs.
-    topk_kernel<<<dim3(G, static_cast<unsigned>(H)), scores ? kTopkThreads : kTopkCandThreads, smem, stream>>>(a);
-    int st = launch_status();
+    // threads; candidate lists take smaller CTAs, and the last CTA of each
+    // group builds its union.
+    st = launch_pdl(topk_kernel, dim3(G, static_cast<unsigned>(H)), dim3(scores ? kTopkThreads : kTopkCandThreads),
+                    smem, stream, a);
+    if (st || !scores) return st;
+    const size_t usmem = 2 * sizeof(int32_t) * G * k;
+    st = ensure_dynamic_smem(reinterpret_cast<const void*>(union_kernel), usmem);
     if (st) return st;
-    int32_t* fault = nullptr;
-    st = device_fault_word(&fault);
-    if (st) return st;
-    const int upow2 = pow2_at_least(G * k);
-    const size_t usmem = sizeof(int32_t) * upow2;
-    e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(usmem));
-    if (e != cudaSuccess) return cuda_status(e);
-    union_kernel<<<static_cast<unsigned>(H), kTopkThreads, usmem, stream>>>(idx, G, k, upow2, union_idx,
-                                                                          union_count, fault);
-    return launch_status();
+    return launch_pdl(union_kernel, dim3(static_cast<unsigned>(H)), dim3(kTopkThreads), usmem, stream, a);
 }
 
 }  // namespace fathom
