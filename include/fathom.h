@@ -342,7 +342,10 @@ size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k);
  * scores / cand is non-NULL:
  *   scores     DEVICE, fp32 [H][G][n] from a DENSE scan.
  *   cand       DEVICE, the candidate buffer of a CANDIDATE scan with the
- *              same H, G, n, k.
+ *              same H, G, n, k.  The call also uses one counter word of
+ *              each group's header in it (left as it found it), so two
+ *              fathom_topk calls on one candidate buffer must not overlap
+ *              on the GPU.
  *   idx        DEVICE out, int32 [H][G][k].
  *   union_idx  DEVICE out, int32 [H][G*k], ascending, -1 padded.
  *   union_count DEVICE out, int32 [H]: size of each union, or

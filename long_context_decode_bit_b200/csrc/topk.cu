@@ -4,14 +4,18 @@
 // union of a KV head's four lists is what gets fetched).
 //
 // Selection is a three-pass radix select (11 + 11 + 10 bits) over the fp32
-// scores mapped to order-preserving uint32 keys, run by one 1024-thread CTA
-// per query head; it yields the k-th largest key T and how many keys equal
-// to T are taken.  Keys above T are all winners; among keys equal to T the
-// lowest indices win (dense scores are scanned in index order; candidate
-// lists are unordered, so their ties are sorted by index).  The k winners
-// are then sorted by (score desc, index asc) with a shared-memory bitonic
-// sort on 64-bit composite keys.  The same select, over per-thread maxima
-// of the sample scores, picks the candidate threshold tau.
+// scores mapped to order-preserving uint32 keys, run by one CTA per query
+// head; it yields the k-th largest key T and how many keys equal to T are
+// taken.  Keys above T are all winners; among keys equal to T the lowest
+// indices win (dense scores are scanned in index order; candidate lists are
+// unordered, so their ties are sorted by index).  The k winners are sorted
+// by (score desc, index asc) for idx, and by index into the group's slice
+// of union_idx.  The union merges a group's G index-sorted lists pairwise
+// and keeps the first of each run of equal indices: on the candidate path
+// the last of the group's G CTAs to finish does it (a per-group counter in
+// the candidate header), after a dense top-k a second kernel does.  The same
+// select, over per-thread maxima of the sample scores, picks the candidate
+// threshold tau.
 #include "common.cuh"
 #include "select.cuh"
 
