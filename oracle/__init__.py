@@ -56,6 +56,8 @@ def _lib():
         lib.orc_layer_budgets.argtypes = [P, P, I64, I, I, I, I64, P]
         lib.orc_pack_nibbles.restype = I
         lib.orc_pack_nibbles.argtypes = [P, I, I64, I64, I, I64, I64, P, I64]
+        lib.orc_rotate_keys.restype = I
+        lib.orc_rotate_keys.argtypes = [P, I, I64, I64, I, I64, I64, P, P]
         lib.orc_union_attention.restype = I
         lib.orc_union_attention.argtypes = [P, P, I, I64, I64, I, I64, I64, P, I, P, P, I64, ctypes.c_double, P]
         _LIB = lib
@@ -108,6 +110,32 @@ def pack(keys: np.ndarray, nb_stride: int | None = None):
     scales = np.zeros((H, D, nbs), dtype=np.uint16)
     _check(_lib().orc_pack(_ptr(keys), dt, H, n, D, n * D, D, _ptr(planes), _ptr(scales), nbs), "pack")
     return planes, scales
+
+
+def rotate_keys(keys: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """Coordinates y [H][n][D] (float32) of keys [H][n][D] (float32, or uint16
+    bf16 bit patterns) in the basis U [H][D][D] (float32, U[h][d][i] =
+    component d of direction i): y_i = sum_d k_d U[d][i] summed over
+    d = 0..D-1 in order, one fp32 fused multiply-add per step."""
+    keys = np.ascontiguousarray(keys)
+    if keys.dtype == np.float32:
+        dt = 0
+    elif keys.dtype == np.uint16:
+        dt = 1
+    else:
+        raise TypeError("keys must be float32 or uint16 (bf16 bits)")
+    H, n, D = keys.shape
+    U = np.ascontiguousarray(U, dtype=np.float32)
+    if U.shape != (H, D, D):
+        raise ValueError("U must be [H][D][D]")
+    out = np.zeros((H, n, D), dtype=np.float32)
+    _check(_lib().orc_rotate_keys(_ptr(keys), dt, H, n, D, n * D, D, _ptr(U), _ptr(out)), "rotate_keys")
+    return out
+
+
+def pack_rotated(keys: np.ndarray, U: np.ndarray, nb_stride: int | None = None):
+    """The index of the keys' coordinates in the basis U: pack(rotate_keys)."""
+    return pack(rotate_keys(keys, U), nb_stride=nb_stride)
 
 
 def importance(sigma2: np.ndarray, q: np.ndarray) -> np.ndarray:

@@ -42,6 +42,11 @@
  *   orc_pack_nibbles   the same 4-bit codes stored whole, 4 bits per token
  *                      (the fixed-depth scans' 4-bit coordinates of the
  *                      byte-accounting section), 16 tokens per 64-bit word
+ *   orc_rotate_keys    the keys' coordinates in a rotated orthonormal basis
+ *                      (base-choice section: models without QK-norm store
+ *                      keys in the KLT basis), in a fixed single-precision
+ *                      order of fused multiply-adds; orc_pack of them is
+ *                      the rotated index
  */
 #include <math.h>
 #include <stdint.h>
@@ -628,5 +633,43 @@ int orc_layer_budgets(const float* sigma2, const float* q, int64_t H, int G, int
     free(items);
     free(N);
     free(ptr);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Keys in a rotated basis (base-choice section: for a model without    */
+/* QK-norm the planes hold the keys' coordinates in an orthonormal      */
+/* basis of directions u_i, the columns of U, and the queries are       */
+/* rotated to match, so q'.y = q.k).  Coordinate i of key k is           */
+/* y_i = sum_d k_d U[d][i].  So that the codes packed from y are        */
+/* defined bit for bit, the sum has one stated single-precision order:  */
+/* y_i starts at +0 and takes k_d * U[d][i] for d = 0, 1, ..., D-1,     */
+/* each step one IEEE fused multiply-add (C99 fmaf: the exact           */
+/* k_d * U[d][i] + y_i, rounded once to nearest-even binary32).  bf16   */
+/* keys are widened to binary32 exactly.  U is [H][D][D] fp32,          */
+/* U[h][d][i]; out is [H][n][D] fp32, contiguous.                        */
+/* ------------------------------------------------------------------ */
+int orc_rotate_keys(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t stride_h,
+                    int64_t stride_tok, const float* U, float* out)
+{
+    if (!keys || !U || !out || H < 0 || n < 0 || D <= 0) return ORC_EINVAL;
+    float* x = (float*)malloc(sizeof(float) * (size_t)D);
+    if (!x) return ORC_ENOMEM;
+    for (int64_t h = 0; h < H; ++h) {
+        const float* Uh = U + h * (int64_t)D * D;
+        for (int64_t tok = 0; tok < n; ++tok) {
+            for (int d = 0; d < D; ++d) {
+                int64_t off = h * stride_h + tok * stride_tok + d;
+                x[d] = key_dtype == 1 ? (float)orc_bf16_value(((const uint16_t*)keys)[off])
+                                      : ((const float*)keys)[off];
+            }
+            for (int i = 0; i < D; ++i) {
+                float y = 0.0f;
+                for (int d = 0; d < D; ++d) y = fmaf(x[d], Uh[(int64_t)d * D + i], y);
+                out[(h * n + tok) * D + i] = y;
+            }
+        }
+    }
+    free(x);
     return ORC_OK;
 }

@@ -720,3 +720,117 @@ def test_layer_budgets_invariances(orc):
     s2_b[P:2 * P] *= np.float32(16.0)
     assert np.array_equal(orc.layer_budgets(s2_b, q_a, 3, 150), base)
     assert np.all(orc.layer_budgets(s2_a, q_a, 1, 50) == 50)
+
+
+# --------------------------------------------------------------------------
+# Rotated basis (section 基座选择: keys stored as their coordinates in an
+# orthonormal KLT basis, queries rotated to match).  The oracle's rotation
+# y_i = sum_d k_d U[d][i] runs in one stated order of fp32 fused
+# multiply-adds (d ascending from +0), so the codes packed from it are
+# defined bit for bit.
+# --------------------------------------------------------------------------
+def _round_f32(x: Fraction) -> Fraction:
+    """Nearest-even binary32 value of the exact rational x (normal and
+    subnormal range; no overflow), by integer arithmetic."""
+    if x == 0:
+        return Fraction(0)
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fraction(2) ** (max(e, -126) - 23)
+    return sign * round(a / quantum) * quantum   # round() on a Fraction is half-to-even
+
+
+def _fma_chain(x, u):
+    y = Fraction(0)
+    for xd, ud in zip(x, u):
+        y = _round_f32(Fraction(float(xd)) * Fraction(float(ud)) + y)
+    return y
+
+
+def test_rotation_identity_and_permutation(orc):
+    rng = np.random.default_rng(11)
+    H, n, D = 2, 150, 32
+    k = (rng.standard_normal((H, n, D)) * np.exp2(rng.integers(-3, 4, (H, 1, D)))).astype(np.float32)
+    kb = (k.view(np.uint32) >> 16).astype(np.uint16)        # bf16 bit patterns (truncated values)
+    eye = np.stack([np.eye(D, dtype=np.float32)] * H)
+    for keys in (k, kb):
+        assert np.array_equal(orc.rotate_keys(keys, eye), orc.rotate_keys(keys, eye))
+        p0, s0 = orc.pack(keys)
+        p1, s1 = orc.pack_rotated(keys, eye)
+        assert np.array_equal(p0, p1) and np.array_equal(s0, s1)
+    assert np.array_equal(orc.rotate_keys(k, eye), k)
+    # U[d][i] = 1 iff d = pi(i): coordinate i is channel pi(i), exactly, and
+    # so are its planes and scales (pi is not an involution: U and U^T differ).
+    pi = np.roll(np.arange(D), 5)
+    P = np.zeros((H, D, D), np.float32)
+    P[:, pi, np.arange(D)] = 1.0
+    assert not np.array_equal(P[0], P[0].T)
+    y = orc.rotate_keys(k, P)
+    assert np.array_equal(y, k[:, :, pi])
+    p0, s0 = orc.pack(k)
+    p1, s1 = orc.pack_rotated(k, P)
+    assert np.array_equal(p1, p0[:, pi]) and np.array_equal(s1, s0[:, pi])
+
+
+def test_rotation_is_the_stated_fma_chain_exactly(orc):
+    # Random inputs against the chain evaluated in exact rational arithmetic
+    # with nearest-even rounding after every step.
+    rng = np.random.default_rng(12)
+    H, n, D = 1, 4, 8
+    k = rng.standard_normal((H, n, D)).astype(np.float32)
+    U = rng.standard_normal((H, D, D)).astype(np.float32)
+    y = orc.rotate_keys(k, U)
+    for t in range(n):
+        for i in range(D):
+            assert Fraction(float(y[0, t, i])) == _fma_chain(k[0, t], U[0, :, i]), (t, i)
+    # Fused: k = (1, a), column (-(1 + 2^-11), a) with a = 1 + 2^-12.  The
+    # exact a*a = 1 + 2^-11 + 2^-24 survives one rounding after the add
+    # (2^-24); a separately rounded product would have given 0.
+    a = 1.0 + 2.0 ** -12
+    U2 = np.zeros((1, 2, 2), np.float32)
+    U2[0, :, 0] = [-(1.0 + 2.0 ** -11), a]
+    y2 = orc.rotate_keys(np.array([[[1.0, a]]], np.float32), U2)
+    assert y2[0, 0, 0] == np.float32(2.0 ** -24)
+    # Order: d ascending.  (2^-30, 1, -1) against a column of ones gives 0
+    # (2^-30 is lost against 1); the reverse order would keep 2^-30.
+    U3 = np.zeros((1, 3, 3), np.float32)
+    U3[0, :, 0] = 1.0
+    y3 = orc.rotate_keys(np.array([[[2.0 ** -30, 1.0, -1.0]]], np.float32), U3)
+    assert y3[0, 0, 0] == 0.0
+    assert _fma_chain([-1.0, 1.0, 2.0 ** -30], [1.0, 1.0, 1.0]) == Fraction(2) ** -30
+
+
+def test_rotated_scores_preserve_q_dot_k(orc):
+    # An orthonormal U keeps q.k: with the queries rotated the same way, the
+    # full-depth scan of the rotated index is q.k up to the quantiser's
+    # half-cell error per coordinate (s/16 in the block's scale) and U's fp32
+    # rounding.  The transposed basis does not: the pin sees the orientation.
+    rng = np.random.default_rng(13)
+    H, n, D, G = 2, 256, 32, 2
+    k = rng.standard_normal((H, n, D)).astype(np.float32)
+    q = rng.standard_normal((H, G, D))
+    U64 = np.stack([np.linalg.qr(rng.standard_normal((D, D)))[0] for _ in range(H)])
+    U = U64.astype(np.float32)
+    exact = np.einsum("hgd,hnd->hgn", q, k.astype(np.float64))
+    full = np.full((H, D), 4, np.uint8)
+
+    def err_and_bound(Uk, Uq):
+        planes, scales = orc.pack_rotated(k, Uk)
+        qr = np.einsum("hgd,hdi->hgi", q, Uq.astype(np.float64)).astype(np.float32)
+        sc = orc.scan(planes, scales, full, qr, n, with_l1=False)
+        s = np.array([[[orc.fp16_value(int(b)) for b in row] for row in sh] for sh in scales])   # [H][D][nb]
+        s_tok = np.repeat(s, 64, axis=2)[:, :, :n]                                              # [H][D][n]
+        bound = np.einsum("hgi,hin->hgn", np.abs(qr.astype(np.float64)), s_tok) / 16.0
+        bound += 1e-5 * np.linalg.norm(q, axis=2)[:, :, None] * np.linalg.norm(k, axis=2)[:, None, :]
+        return np.abs(sc - exact), bound
+
+    err, bound = err_and_bound(U, U)
+    assert np.all(err <= bound)
+    # Keys rotated by U^T while the queries use U: the bound fails widely.
+    err_t, bound_t = err_and_bound(np.ascontiguousarray(U.transpose(0, 2, 1)), U)
+    assert np.mean(err_t > bound_t) > 0.1
