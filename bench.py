@@ -293,7 +293,7 @@ def run_gpu(args):
         f"{(planes.numel() * 8 + scales.numel() * 2) / 1e9:.2f} GB")
 
     step = fathom.Step(planes, scales, w.n, sigma2, w.G, k, budget=B)
-    launches_per_step = 6   # plan, sample scan, tau, filter scan, top-k, union
+    launches_per_step = 5   # plan, sample scan, tau, filter scan, top-k (the union runs inside it)
 
     def one(ev):
         step.run_plan(q)
@@ -382,7 +382,7 @@ def run_gpu(args):
                  "active_channels_range": [min(na), max(na)]},
         "e2e": {"value": keys_per_step / (e2e_ms / 1e3), "unit": "keys/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps + (2 * fallback * args.steps if fallback else 0),
+        "gpu_launches": launches_per_step * args.steps + (3 * fallback * args.steps if fallback else 0),
         "clocks": clocks, "pack": pack, "fallback_groups": fallback, "overflow_after_timing": bad_after,
     }
     if sweep is not None:
@@ -678,7 +678,60 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
             st.run(ql, check_overflow=False)
     seq(None)
     tot, _ = time_steps(seq, 5, 2, device)
-    out["per_layer_B48"] = {"layers": layers, "groups_per_layer": per, "ms_per_step": tot / 5}
+    # The same launches replayed from a CUDA graph (no host issue cost).
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(side):
+        seq(None)
+    torch.cuda.current_stream(device).wait_stream(side)
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        seq(None)
+    tg, _ = time_steps(lambda ev: graph.replay(), 5, 2, device)
+    del graph
+    out["per_layer_B48"] = {"layers": layers, "groups_per_layer": per, "ms_per_step": tot / 5,
+                            "ms_per_step_graph": tg / 5, "launches_per_layer": 5}
+    del steps
+    out["host_resident_1M"] = host_resident_entry(w, planes, scales, sigma2, q, k, device, log)
+    return out
+
+
+def host_resident_entry(w, planes, scales, sigma2, q, k, device, log):
+    """One session of the step's index (288 groups x 2^20 tokens, about 20 GB)
+    in page-locked host memory, scanned zero-copy over the host link at B = 48
+    and B = 136; bytes read per step against the measured H2D bandwidth
+    (best of 10), with the clocks of the timed region."""
+    import torch
+    from long_context_decode_bit_b200 import fathom
+    t0 = time.time()
+    hp = torch.empty(planes.shape, dtype=planes.dtype, pin_memory=True)
+    hs = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+    hp.copy_(planes)
+    hs.copy_(scales)
+    pinned_gb = (hp.numel() * 8 + hs.numel() * 2) / 1e9
+    log(f"[bench] host-resident session: {pinned_gb:.1f} GB pinned in {time.time() - t0:.0f}s")
+    link = h2d_bandwidth(device)
+    props = torch.cuda.get_device_properties(device)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(device.index or 0)
+    out = {"workload": w.name, "pinned_GB": pinned_gb, "h2d_GBps_best_of_10": link}
+    for bname, bb in (("B48", 48), ("B136", 136)):
+        st = fathom.Step(hp, hs, w.n, sigma2, w.G, k, budget=bb)
+
+        def one(ev, st=st):
+            st.run(q, check_overflow=False)
+        one(None)
+        torch.cuda.synchronize(device)
+        fb = st.repair(q)
+        alg = plan_bytes(st, w)[0]
+        with ClockSampler(gpu_id) as clk:
+            tot, _ = time_steps(one, 3, 1, device)
+        ms = tot / 3
+        out[bname] = {"ms_per_step": ms, "keys_per_s": w.H * w.n / (ms / 1e3), "alg_bytes": alg,
+                      "read_bits_per_token": alg * 8 / (w.H * w.n), "link_GBps": alg / (ms / 1e3) / 1e9,
+                      "link_frac": alg / (ms / 1e3) / 1e9 / link, "fallback_groups": fb, "clocks": clk.summary()}
+        del st
+    del hp, hs
     return out
 
 
