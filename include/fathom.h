@@ -119,6 +119,30 @@ int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
                 fathom_stream_t stream);
 
 /*
+ * fathom_pack_rotated -- the index of the keys' coordinates in an
+ * orthonormal basis U (基座选择: for models without QK-norm the planes hold
+ * each key in the KLT basis of the calibration keys, and the queries are
+ * rotated the same way, q'_i = sum_d q_d U[d][i], so q'.y = q.k).  Equal to
+ * fathom_pack of the rotated keys y [H][n][D], which are never written:
+ *   y_i = sum_d k_d U[h][d][i], summed over d = 0, 1, ..., D-1 in that order
+ *   from +0, every step one fp32 fused multiply-add (one rounding).
+ * The order is part of the definition: the planes are bit-exact against any
+ * evaluation of the same chain.
+ *
+ *   keys, key_dtype, H, n, D, key strides, planes, scales, nb_stride
+ *               as for fathom_pack (keys finite; the rotated coordinates
+ *               must stay below 65520 in magnitude).
+ *   U           DEVICE, fp32 [H][D][D], contiguous: U[(h*D + d)*D + i] is
+ *               component d of direction i (columns are the directions).
+ * Cost: D fused multiply-adds per coordinate per token (FP32-pipe bound).
+ * Appending works as for fathom_pack (rewrite from the tail block on).
+ */
+int fathom_pack_rotated(const void* keys, int key_dtype, int64_t H, int64_t n, int D,
+                        int64_t key_stride_h, int64_t key_stride_tok, const float* U,
+                        uint64_t* planes, uint16_t* scales, int64_t nb_stride,
+                        fathom_stream_t stream);
+
+/*
  * fathom_calibrate_workspace_bytes -- scratch fathom_calibrate needs (HOST
  * call); 0 for unsupported sizes.
  */

@@ -13,6 +13,9 @@ namespace fathom {
 
 int launch_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t stride_h,
                 int64_t stride_tok, uint64_t* planes, uint16_t* scales, int64_t nb_stride, cudaStream_t stream);
+int launch_pack_rotated(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t stride_h,
+                        int64_t stride_tok, const float* U, uint64_t* planes, uint16_t* scales, int64_t nb_stride,
+                        cudaStream_t stream);
 int launch_plan(const float* sigma2, const float* q, int64_t H, int G, int D, const int32_t* budget_bits,
                 int32_t budget_flat, uint8_t* depth, uint16_t* active, int32_t* n_active, float* theta,
                 cudaStream_t stream);
@@ -223,6 +226,30 @@ int fathom_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, in
     FATHOM_TRY(check_device_ptr(scales));
     return launch_pack(keys, key_dtype, H, n, D, key_stride_h, key_stride_tok, planes, scales, nb_stride,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fathom_pack_rotated(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t key_stride_h,
+                        int64_t key_stride_tok, const float* U, uint64_t* planes, uint16_t* scales,
+                        int64_t nb_stride, fathom_stream_t stream)
+{
+    NvtxRange range("fathom_pack_rotated");
+    if (H < 0 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
+    if (key_dtype != FATHOM_KEYS_F32 && key_dtype != FATHOM_KEYS_BF16) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
+    if (H == 0 || n == 0) return FATHOM_OK;
+    const int64_t nb = ceil_div(n, kBlockTokens);
+    if (nb_stride < nb || (nb_stride & 1)) return FATHOM_ERR_INVALID_ARG;
+    if (key_stride_tok < D || (H > 1 && key_stride_h < n * key_stride_tok)) return FATHOM_ERR_INVALID_ARG;
+    if (H * (D % 128 == 0 ? D / 128 : (D % 64 == 0 ? D / 64 : D / 32)) > 65535) return FATHOM_ERR_UNSUPPORTED;
+    if (!aligned(planes, 8) || !aligned(scales, 2) || !aligned(U, 4) ||
+        !aligned(keys, key_dtype == FATHOM_KEYS_F32 ? 4 : 2))
+        return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(keys));
+    FATHOM_TRY(check_device_ptr(U));
+    FATHOM_TRY(check_device_ptr(planes));
+    FATHOM_TRY(check_device_ptr(scales));
+    return launch_pack_rotated(keys, key_dtype, H, n, D, key_stride_h, key_stride_tok, U, planes, scales, nb_stride,
+                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fathom_layer_budgets_workspace_bytes(int64_t H, int D)

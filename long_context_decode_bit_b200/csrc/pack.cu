@@ -103,7 +103,166 @@ pack_kernel(const T* __restrict__ keys, int64_t H, int64_t n, int D, int64_t str
     }
 }
 
+// ---------------------------------------------------------------------
+// fathom_pack_rotated: the index of the keys' coordinates in an orthonormal
+// basis U (Fathom, section 基座选择: for models without QK-norm the keys
+// are stored in the KLT basis and the queries rotated to match).
+// Coordinate i of key k is y_i = sum_d k_d U[d][i], accumulated in fp32
+// fused multiply-adds in the order d = 0, 1, ..., D-1 from +0: the order is
+// part of the definition, so the codes are bit-exact against any evaluation
+// of the same chain.  The rotated keys never reach device memory.
+//
+// One CTA owns C output coordinates of one group and walks the group's
+// 64-token blocks; its D x C slice of U stays in shared memory.  Each
+// block's keys are staged channel-major (a row of 64 tokens per channel).
+// Warp w owns coordinates [w*C/8, (w+1)*C/8); a lane accumulates TOK
+// consecutive tokens of one coordinate in registers (float4 reads of the
+// staged keys, one U value per step), then quantises them exactly as
+// fathom_pack does: the block maximum over the lanes that share the
+// coordinate, the fp16 scale, the codes, and each lane's TOK bits of every
+// plane word, joined by shuffles.  Cost: D fused multiply-adds per output
+// coordinate per token, so the kernel is bound by the FP32 pipe, not HBM.
+// ---------------------------------------------------------------------
+constexpr int kRotThreads = 256;
+constexpr int kRotRow = kBlockTokens + 4;   // staged key row: 64 tokens + pad (16-byte multiple)
+
+template <int C>
+size_t rot_smem_bytes(int D)
+{
+    return sizeof(float) * (static_cast<size_t>(D) * C + static_cast<size_t>(D) * kRotRow);
+}
+
+template <typename T, int C>
+__global__ void __launch_bounds__(kRotThreads)
+pack_rotated_kernel(const T* __restrict__ keys, int64_t n, int D, int64_t stride_h, int64_t stride_tok,
+                    const float* __restrict__ U, uint64_t* __restrict__ planes, uint16_t* __restrict__ scales,
+                    int64_t nb_stride, int64_t nb)
+{
+    constexpr int OPW = C / 8;                  // coordinates per warp
+    constexpr int TOK = kBlockTokens * OPW / 32; // tokens per lane
+    extern __shared__ __align__(16) float rsm[];
+    float* Us = rsm;                            // [D][C]
+    float* Xs = rsm + static_cast<size_t>(D) * C;   // [D][kRotRow]
+
+    const int chunks = D / C;
+    const int64_t h = blockIdx.y / chunks;
+    const int c0 = (blockIdx.y % chunks) * C;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cl = warp * OPW + lane % OPW;     // coordinate of the lane within the chunk
+    const int qg = lane / OPW;                  // token group of the lane
+    const int tok0 = qg * TOK;
+
+    const float* Uh = U + h * static_cast<int64_t>(D) * D;
+    for (int i = tid; i < D * C; i += kRotThreads) Us[i] = Uh[static_cast<int64_t>(i / C) * D + c0 + i % C];
+    const T* kh = keys + h * stride_h;
+    const int j = c0 + cl;
+
+    for (int64_t b = blockIdx.x; b < nb; b += gridDim.x) {
+        const int64_t t0 = b * kBlockTokens;
+        __syncthreads();   // the previous block's keys are no longer read (and U is staged)
+        for (int i = tid; i < kBlockTokens * D; i += kRotThreads) {
+            const int t = i / D, d = i % D;
+            Xs[d * kRotRow + t] = (t0 + t < n) ? load_key(kh + (t0 + t) * stride_tok + d) : 0.0f;
+        }
+        __syncthreads();
+
+        float acc[TOK];
+#pragma unroll
+        for (int t = 0; t < TOK; ++t) acc[t] = 0.0f;
+#pragma unroll 2
+        for (int d = 0; d < D; ++d) {
+            const float u = Us[d * C + cl];
+            const float4* xr = reinterpret_cast<const float4*>(Xs + d * kRotRow + tok0);
+#pragma unroll
+            for (int v = 0; v < TOK / 4; ++v) {
+                const float4 x = xr[v];
+                acc[4 * v + 0] = fmaf(x.x, u, acc[4 * v + 0]);
+                acc[4 * v + 1] = fmaf(x.y, u, acc[4 * v + 1]);
+                acc[4 * v + 2] = fmaf(x.z, u, acc[4 * v + 2]);
+                acc[4 * v + 3] = fmaf(x.w, u, acc[4 * v + 3]);
+            }
+        }
+
+        // Block maximum over the valid tokens, across the lanes of this coordinate.
+        float m = 0.0f;
+#pragma unroll
+        for (int t = 0; t < TOK; ++t)
+            if (t0 + tok0 + t < n) m = fmaxf(m, fabsf(acc[t]));
+#pragma unroll
+        for (int o = OPW; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const __half s16 = __float2half_rn(m);
+        const float s = __half2float(s16);
+        uint32_t piece[kPlanes] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int t = 0; t < TOK; ++t) {
+            if (t0 + tok0 + t >= n) continue;
+            const int c = code4(acc[t], s);
+#pragma unroll
+            for (int p = 0; p < kPlanes; ++p) piece[p] |= static_cast<uint32_t>((c >> (3 - p)) & 1) << t;
+        }
+        // Join the 64 / TOK pieces of each plane word (token group g at bit g*TOK).
+        uint64_t word[kPlanes] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int g = 0; g < 32 / OPW; ++g)
+#pragma unroll
+            for (int p = 0; p < kPlanes; ++p)
+                word[p] |= static_cast<uint64_t>(__shfl_sync(0xffffffffu, piece[p], lane % OPW + g * OPW))
+                           << (g * TOK);
+        if (qg == 0) {
+            const int64_t row = (h * D + j) * kPlanes;
+#pragma unroll
+            for (int p = 0; p < kPlanes; ++p) planes[(row + p) * nb_stride + b] = word[p];
+            scales[(h * D + j) * nb_stride + b] = __half_as_ushort(s16);
+        }
+    }
+}
+
+template <typename T, int C>
+int launch_pack_rotated_t(const T* keys, int64_t H, int64_t n, int D, int64_t stride_h, int64_t stride_tok,
+                          const float* U, uint64_t* planes, uint16_t* scales, int64_t nb_stride,
+                          cudaStream_t stream)
+{
+    const size_t smem = rot_smem_bytes<C>(D);
+    int st = ensure_dynamic_smem(reinterpret_cast<const void*>(pack_rotated_kernel<T, C>), smem);
+    if (st) return st;
+    int sms = 0;
+    st = device_sm_count(&sms);
+    if (st) return st;
+    const int64_t nb = ceil_div(n, kBlockTokens);
+    const int64_t rows = H * (D / C);
+    const int per_sm = smem <= 110 * 1024 ? 2 : 1;
+    int64_t gx = ceil_div(static_cast<int64_t>(sms) * per_sm * 2, rows);   // about two waves of CTAs
+    gx = gx < 1 ? 1 : (gx > nb ? nb : gx);
+    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(rows));
+    pack_rotated_kernel<T, C><<<grid, kRotThreads, smem, stream>>>(keys, n, D, stride_h, stride_tok, U, planes,
+                                                                   scales, nb_stride, nb);
+    return launch_status();
+}
+
+template <typename T>
+int launch_pack_rotated_c(const T* keys, int64_t H, int64_t n, int D, int64_t stride_h, int64_t stride_tok,
+                          const float* U, uint64_t* planes, uint16_t* scales, int64_t nb_stride,
+                          cudaStream_t stream)
+{
+    if (D % 128 == 0)
+        return launch_pack_rotated_t<T, 128>(keys, H, n, D, stride_h, stride_tok, U, planes, scales, nb_stride, stream);
+    if (D % 64 == 0)
+        return launch_pack_rotated_t<T, 64>(keys, H, n, D, stride_h, stride_tok, U, planes, scales, nb_stride, stream);
+    return launch_pack_rotated_t<T, 32>(keys, H, n, D, stride_h, stride_tok, U, planes, scales, nb_stride, stream);
+}
+
 }  // namespace
+
+int launch_pack_rotated(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t stride_h,
+                        int64_t stride_tok, const float* U, uint64_t* planes, uint16_t* scales, int64_t nb_stride,
+                        cudaStream_t stream)
+{
+    if (key_dtype == FATHOM_KEYS_F32)
+        return launch_pack_rotated_c(static_cast<const float*>(keys), H, n, D, stride_h, stride_tok, U, planes,
+                                     scales, nb_stride, stream);
+    return launch_pack_rotated_c(static_cast<const __nv_bfloat16*>(keys), H, n, D, stride_h, stride_tok, U, planes,
+                                 scales, nb_stride, stream);
+}
 
 int launch_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, int64_t stride_h,
                 int64_t stride_tok, uint64_t* planes, uint16_t* scales, int64_t nb_stride,

@@ -40,7 +40,7 @@ EXPORTS = (
     "fathom_device_status", "fathom_calibrate_workspace_bytes", "fathom_calibrate",
     "fathom_union_attention_workspace_bytes", "fathom_union_attention",
     "fathom_nibbles_from_planes", "fathom_scan_nibbles", "fathom_layer_budgets_workspace_bytes",
-    "fathom_layer_budgets",
+    "fathom_layer_budgets", "fathom_pack_rotated",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -84,6 +84,7 @@ def load(path: str | None = None):
         "fathom_dequant_rows": (I, [P, P, I64, I, I64, I64, P, I64, P, I, P, P]),
         "fathom_scan_topk_noalloc": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, P, P]),
         "fathom_device_status": (I, [I, P]),
+        "fathom_pack_rotated": (I, [P, I, I64, I64, I, I64, I64, P, P, P, I64, P]),
         "fathom_calibrate_workspace_bytes": (SZ, [I64, I, I]),
         "fathom_calibrate": (I, [P, I, I64, I64, I, I64, I64, P, P, P, P, SZ, P]),
         "fathom_union_attention_workspace_bytes": (SZ, [I64, I, I, I64]),
@@ -146,6 +147,28 @@ def pack(keys: torch.Tensor, nb_stride_words: int | None = None, planes=None, sc
         scales = torch.zeros((H, D, nbs), dtype=torch.int16, device=dev)
     _check(lib().fathom_pack(_p(keys), dt, H, n, D, keys.stride(0), keys.stride(1), _p(planes), _p(scales),
                              nbs, _stream(stream)), "fathom_pack")
+    return planes, scales
+
+
+def pack_rotated(keys: torch.Tensor, U: torch.Tensor, nb_stride_words: int | None = None, planes=None, scales=None,
+                 stream=None):
+    """Bit-plane index of the keys' coordinates in the basis U [H][D][D]
+    (fp32, columns = directions), rotated inside the kernel in a fixed fp32
+    fused multiply-add order (see fathom_pack_rotated in include/fathom.h)."""
+    H, n, D = keys.shape
+    if keys.stride(2) != 1:
+        raise ValueError("keys must be contiguous along channels")
+    if U.dtype != torch.float32 or tuple(U.shape) != (H, D, D) or not U.is_contiguous():
+        raise ValueError("U must be a contiguous fp32 [H][D][D] tensor")
+    dt = {torch.float32: KEYS_F32, torch.bfloat16: KEYS_BF16}[keys.dtype]
+    nbs = nb_stride(n) if nb_stride_words is None else int(nb_stride_words)
+    dev = keys.device
+    if planes is None:
+        planes = torch.zeros((H, D, 4, nbs), dtype=torch.int64, device=dev)
+    if scales is None:
+        scales = torch.zeros((H, D, nbs), dtype=torch.int16, device=dev)
+    _check(lib().fathom_pack_rotated(_p(keys), dt, H, n, D, keys.stride(0), keys.stride(1), _p(U), _p(planes),
+                                     _p(scales), nbs, _stream(stream)), "fathom_pack_rotated")
     return planes, scales
 
 

@@ -2,6 +2,7 @@
 same seeded inputs.  Planes, scales and plans must be bit-exact; scores
 within 1e-5 of their L1 scale; top-k sets equal up to ties at the k-th
 score; top-k of the GPU's own scores identical to a full sort of them."""
+import ctypes
 import dataclasses
 
 import numpy as np
@@ -556,3 +557,49 @@ def test_nibble_scan_other_shapes(fathom_gpu, orc, D, G):
     s_pl = fathom_gpu.scan(planes, scales, w.n, active, na, q)
     torch.cuda.synchronize()
     assert torch.equal(s_nib, s_pl)
+
+
+# --------------------------------------------------------------------------
+# Fused KLT rotation inside pack (section 基座选择): bit-exact planes and
+# scales against the oracle's fixed-order fp32 fused multiply-add chain.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("D,n,dtype", [(128, 3000, torch.bfloat16), (128, 64 * 37, torch.float32),
+                                       (64, 1000, torch.bfloat16), (96, 777, torch.float32),
+                                       (256, 700, torch.bfloat16)],
+                         ids=["d128-bf16-ragged", "d128-f32", "d64-bf16", "d96-f32", "d256-bf16"])
+def test_pack_rotated_matches_oracle(fathom_gpu, orc, D, n, dtype):
+    from long_context_decode_bit_b200 import basis
+    w = dataclasses.replace(inputs.LAYER_32K, name=f"rot-{D}-{n}", H=3, n=n, D=D, kind="corr", n_cal=min(n, 512), seed=77 + D)
+    k = inputs.keys(w, 0, w.H, device=DEV).to(dtype).contiguous()
+    q = inputs.queries(w, 0, w.H, device=DEV).float().contiguous()
+    U = basis.klt_basis(k[:, :w.n_cal], q).contiguous()
+    planes, scales = fathom_gpu.pack_rotated(k, U)
+    torch.cuda.synchronize()
+    p_ref, s_ref = orc.pack_rotated(keys_for_oracle(k), U.cpu().numpy(), nb_stride=planes.shape[-1])
+    assert np.array_equal(np_u64(planes), p_ref)
+    assert np.array_equal(np_u16(scales), s_ref)
+
+
+def test_pack_rotated_identity_is_pack_and_appends(fathom_gpu):
+    w = dataclasses.replace(inputs.LAYER_32K, name="rot-eye", H=2, n=5000, seed=78)
+    k = inputs.keys(w, 0, w.H, device=DEV)
+    eye = torch.eye(w.D, device=DEV).expand(w.H, w.D, w.D).contiguous()
+    p0, s0 = fathom_gpu.pack(k)
+    p1, s1 = fathom_gpu.pack_rotated(k, eye)
+    torch.cuda.synchronize()
+    assert torch.equal(p0, p1) and torch.equal(s0, s1)
+    # Rewriting from block b0 on (the decode-time append) equals packing at once.
+    U = torch.linalg.qr(torch.randn(w.H, w.D, w.D, device=DEV, dtype=torch.float64))[0].float().contiguous()
+    pa, sa = fathom_gpu.pack_rotated(k, U)
+    b0 = 40
+    pb = torch.zeros_like(pa)
+    sb = torch.zeros_like(sa)
+    fathom_gpu.pack_rotated(k[:, :64 * b0 + 10].contiguous(), U, nb_stride_words=pa.shape[-1], planes=pb, scales=sb)
+    lib = fathom_gpu.lib()
+    tail = k[:, 64 * b0:].contiguous()
+    st = lib.fathom_pack_rotated(fathom_gpu._p(tail), fathom_gpu.KEYS_BF16, w.H, tail.shape[1], w.D, tail.stride(0),
+                                 tail.stride(1), fathom_gpu._p(U), ctypes.c_void_p(pb.data_ptr() + 8 * b0),
+                                 ctypes.c_void_p(sb.data_ptr() + 2 * b0), pa.shape[-1], fathom_gpu._stream(None))
+    assert st == fathom_gpu.OK
+    torch.cuda.synchronize()
+    assert torch.equal(pa, pb) and torch.equal(sa, sb)
