@@ -177,7 +177,7 @@ def alu_roofline(fmas: int, ms: float, clocks: dict, props) -> dict:
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for name in ("scan.cu", "common.cuh"):
+    for name in ("scan.cu", "common.cuh", "ring.cuh"):
         with open(os.path.join(ROOT, "long_context_decode_bit_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -481,6 +481,14 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     import torch
     from long_context_decode_bit_b200 import fathom
     out = {}
+    hbm_peak, _ = measured_peaks()
+    fma_peak = torch.cuda.get_device_properties(device).multi_processor_count * 128 * 1965e6   # FMA lanes x max clock
+
+    def fracs(moved_bytes, n, G, active, ms):
+        """Filter scan's fraction of measured HBM bandwidth and of the fp32 FMA
+        pipe (G multiply-adds per key per active channel, at the max SM clock)."""
+        return {"hbm_frac": moved_bytes / (ms / 1e3) / 1e9 / hbm_peak,
+                "fma_frac": n * G * sum(active) / (ms / 1e3) / fma_peak}
     variants = [(f"B{b}", dict(budget=b)) for b in (48, 68, 92, 136)] + [
         ("fixed136_r32", dict(fixed_r=32)),                        # 32 channels x 4 bits + scales
         ("sparq68_r16", dict(fixed_r=16)),                         # 16 channels x 4 bits + scales
@@ -505,7 +513,8 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
         fm = statistics.fmean(fk)
         out[name] = {"ms_per_step": tot / 5, "scan_ms": fm, "scan_GBps": alg / (fm / 1e3) / 1e9,
                      "read_bits_per_token": alg * 8 / (w.H * w.n), "plane_bits_mean": statistics.fmean(bits),
-                     "active_channels_mean": statistics.fmean(na), "fallback_groups": fb}
+                     "active_channels_mean": statistics.fmean(na), "fallback_groups": fb,
+                     **fracs(alg, w.n, w.G, na, fm)}
         del st
     # The rotated-basis run on the Llama-3.1-8B shape (32 layers x 8 KV heads).
     from long_context_decode_bit_b200 import inputs as _inputs
@@ -535,7 +544,7 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
             out[bname] = {"workload": wl.name, "ms_per_step": tot / 5, "scan_ms": fm,
                           "scan_GBps": alg / (fm / 1e3) / 1e9, "keys_per_s": wl.H * wl.n / (tot / 5 / 1e3),
                           "read_bits_per_token": alg * 8 / (wl.H * wl.n), "active_channels_mean": statistics.fmean(na),
-                          "fallback_groups": fb}
+                          "fallback_groups": fb, **fracs(alg, wl.n, wl.G, na, fm)}
             del st
         del rp, rs
         torch.cuda.empty_cache()
@@ -612,8 +621,39 @@ def run_sweep(w, planes, scales, sigma2, q, k, device, log):
     tot, fk = time_steps(onen, 5, 2, device, kernel_events=True)
     fm = statistics.fmean(fk)
     out["nibble136_r32"] = {"ms_per_step": tot / 5, "scan_ms": fm, "scan_GBps": alg / (fm / 1e3) / 1e9,
-                            "read_bits_per_token": alg * 8 / (w.H * w.n), "fallback_groups": fbn}
+                            "read_bits_per_token": alg * 8 / (w.H * w.n), "fallback_groups": fbn,
+                            **fracs(alg, w.n, w.G, na, fm)}
     del stn, nib
+    torch.cuda.empty_cache()
+    # The same scan over a token-major 4-bit copy (one D/2-byte row per token,
+    # as a serving stack keeps a 4-bit K cache): whole rows move.
+    from long_context_decode_bit_b200 import accounting as _acc
+    tm = fathom.nibbles_tm_from_planes(planes, w.n)
+    stt = fathom.Step(planes, scales, w.n, sigma2, w.G, k, fixed_r=32, nibbles=tm, token_major=True)
+
+    def onet(ev, st=stt):
+        st.run_plan(q)
+        st.run_prepare(q)
+        if ev is not None:
+            ev[0].record()
+        st.run_filter(q)
+        if ev is not None:
+            ev[1].record()
+        st.run_topk()
+    onet(None)
+    torch.cuda.synchronize(device)
+    fbt = stt.repair(q)
+    na_t = stt.plan_out[2].to("cpu").tolist()
+    alg_t = sum(_acc.token_major_scan_bytes(w.n, int(a), w.G, w.D) for a in na_t)
+    useful = plan_bytes(stt, w)[0]
+    tot, fk = time_steps(onet, 5, 2, device, kernel_events=True)
+    fm = statistics.fmean(fk)
+    out["nibble136_tm_r32"] = {"ms_per_step": tot / 5, "scan_ms": fm, "scan_GBps": alg_t / (fm / 1e3) / 1e9,
+                               "moved_bits_per_token": alg_t * 8 / (w.H * w.n),
+                               "useful_bits_per_token": useful * 8 / (w.H * w.n),
+                               "store_bytes_per_token_per_kv_head": w.D // 2, "fallback_groups": fbt,
+                               **fracs(alg_t, w.n, w.G, na_t, fm)}
+    del stt, tm
     torch.cuda.empty_cache()
     # Attention of the step's query heads over their union rows, for the
     # first layer's 8 groups (their full-precision K/V cache regenerated).

@@ -352,6 +352,38 @@ int fathom_scan_nibbles(const uint64_t* nibbles, const uint16_t* scales, int64_t
                         fathom_stream_t stream);
 
 /*
+ * fathom_nibbles_tm_from_planes -- the same 4-bit codes stored TOKEN-MAJOR,
+ * as a serving stack keeps a 4-bit K cache: token i of group h owns one row
+ * of D/2 bytes, byte c holding channel 2c in its low nibble and channel
+ * 2c + 1 in its high nibble:
+ *   store[(h * 64 * nb_stride + i) * (D/2) + c],
+ * rows for tokens 0 .. 64*ceil(n/64) - 1 written (tokens past n hold code
+ * 0).  Scales stay the planes' own.  A scan of r chosen channels moves whole
+ * rows: D/2 bytes per token per KV head (64 B at D = 128) whatever r is,
+ * against r/2 bytes in the channel-major stores (先算一笔字节账: the
+ * fixed-depth scans' 4-bit coordinates).
+ *
+ *   planes      DEVICE, as written by fathom_pack.
+ *   store       DEVICE out, uint8 [H][64*nb_stride][D/2], 16-byte aligned.
+ */
+int fathom_nibbles_tm_from_planes(const uint64_t* planes, int64_t H, int D, int64_t n,
+                                  int64_t nb_stride, uint8_t* store, fathom_stream_t stream);
+
+/*
+ * fathom_scan_nibbles_tm -- fathom_scan_nibbles over the token-major store:
+ * every active channel read at 4 bits, value (c - 7.5) s/8 with the
+ * channel's block scale.  Arguments, modes, outputs and errors are
+ * fathom_scan's, with `store` in place of `planes` (the candidate buffer
+ * and fathom_topk are shared).  Scores agree with fathom_scan_nibbles to
+ * fp32 rounding (the sums run in another order).
+ */
+int fathom_scan_nibbles_tm(const uint8_t* store, const uint16_t* scales, int64_t H, int D,
+                           int64_t n, int64_t nb_stride, const uint16_t* active,
+                           const int32_t* n_active, const float* q, int G, int mode,
+                           float* scores, void* cand, size_t cand_bytes, int k,
+                           fathom_stream_t stream);
+
+/*
  * fathom_topk_workspace_bytes -- scratch fathom_topk needs (HOST call).
  */
 size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k);

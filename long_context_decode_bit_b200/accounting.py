@@ -43,6 +43,17 @@ def scan_bytes(n: int, plane_bits: int, n_active: int, G: int = 4, D: int = 128,
     return b
 
 
+def token_major_scan_bytes(n: int, n_active: int, G: int = 4, D: int = 128, query_bytes: bool = True) -> int:
+    """Bytes one group's scan of a token-major 4-bit copy moves: whole rows
+    of D/2 bytes per token (whatever the number of channels read) plus one
+    2-byte scale per active channel per block and the group's queries."""
+    nb = (n + BLOCK - 1) // BLOCK
+    b = n * D // 2 + n_active * 2 * nb
+    if query_bytes:
+        b += G * D * 4
+    return b
+
+
 def step_scan_bytes(n: int, plan_bits, plan_active, G: int = 4, D: int = 128) -> int:
     """Algorithmic bytes over all groups of one step."""
     return sum(scan_bytes(n, int(b), int(a), G, D) for b, a in zip(plan_bits, plan_active))

@@ -26,6 +26,11 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
                 void* cand, int k, bool nib, cudaStream_t stream);
 int launch_topk(const float* scores, const void* cand, int64_t H, int G, int64_t n, int k, int32_t* idx,
                 int32_t* union_idx, int32_t* union_count, cudaStream_t stream);
+int launch_scan_tm(const uint8_t* store, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
+                   const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
+                   void* cand, int k, cudaStream_t stream);
+int launch_tm_from_planes(const uint64_t* planes, int64_t H, int D, int64_t n, int64_t nb_stride, uint8_t* store,
+                          cudaStream_t stream);
 
 int launch_dequant_rows(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n,
                         int64_t nb_stride, const int32_t* rows, int64_t M, const int32_t* row_count, int bits,
@@ -94,9 +99,12 @@ bool dims_ok(int D, int G) { return D >= 32 && D <= kMaxD && D % 32 == 0 && G >=
         if (_st != FATHOM_OK) return _st; \
     } while (0)
 
-int scan_entry(const uint64_t* planes, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
+// Store layouts a scan reads: bit planes, channel-major nibbles, token-major nibble rows.
+enum StoreLayout { kPlanesLayout = 0, kNibblesLayout = 1, kTokenMajorLayout = 2 };
+
+int scan_entry(const void* planes, const uint16_t* scales, int64_t H, int D, int64_t n, int64_t nb_stride,
                const uint16_t* active, const int32_t* n_active, const float* q, int G, int mode, float* scores,
-               void* cand, size_t cand_bytes, int k, bool nib, fathom_stream_t stream)
+               void* cand, size_t cand_bytes, int k, StoreLayout layout, fathom_stream_t stream)
 {
     if (H < 0 || H > 65535 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
     if (!dims_ok(D, G)) return FATHOM_ERR_UNSUPPORTED;
@@ -122,8 +130,11 @@ int scan_entry(const uint64_t* planes, const uint16_t* scales, int64_t H, int D,
         FATHOM_TRY_IN(check_device_ptr(cand));
         if (cand_bytes < cand_layout(H, G, n, k).total) return FATHOM_ERR_WORKSPACE;
     }
-    return launch_scan(planes, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, k, nib,
-                       reinterpret_cast<cudaStream_t>(stream));
+    if (layout == kTokenMajorLayout)
+        return launch_scan_tm(static_cast<const uint8_t*>(planes), scales, H, D, n, nb_stride, active, n_active, q, G,
+                              mode, scores, cand, k, reinterpret_cast<cudaStream_t>(stream));
+    return launch_scan(static_cast<const uint64_t*>(planes), scales, H, D, n, nb_stride, active, n_active, q, G, mode,
+                       scores, cand, k, layout == kNibblesLayout, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // One thread per (group, channel, block): the four plane words -> the four
@@ -395,7 +406,7 @@ int fathom_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
 {
     NvtxRange range("fathom_scan");
     return fathom::scan_entry(planes, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, cand_bytes, k,
-                      false, stream);
+                              fathom::kPlanesLayout, stream);
 }
 
 int fathom_scan_nibbles(const uint64_t* nibbles, const uint16_t* scales, int64_t H, int D, int64_t n,
@@ -404,7 +415,31 @@ int fathom_scan_nibbles(const uint64_t* nibbles, const uint16_t* scales, int64_t
 {
     NvtxRange range("fathom_scan_nibbles");
     return fathom::scan_entry(nibbles, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, cand_bytes, k,
-                      true, stream);
+                              fathom::kNibblesLayout, stream);
+}
+
+int fathom_scan_nibbles_tm(const uint8_t* store, const uint16_t* scales, int64_t H, int D, int64_t n,
+                           int64_t nb_stride, const uint16_t* active, const int32_t* n_active, const float* q, int G,
+                           int mode, float* scores, void* cand, size_t cand_bytes, int k, fathom_stream_t stream)
+{
+    NvtxRange range("fathom_scan_nibbles_tm");
+    return fathom::scan_entry(store, scales, H, D, n, nb_stride, active, n_active, q, G, mode, scores, cand, cand_bytes,
+                              k, fathom::kTokenMajorLayout, stream);
+}
+
+int fathom_nibbles_tm_from_planes(const uint64_t* planes, int64_t H, int D, int64_t n, int64_t nb_stride,
+                                  uint8_t* store, fathom_stream_t stream)
+{
+    NvtxRange range("fathom_nibbles_tm_from_planes");
+    if (H < 0 || n < 0 || n >= (1LL << 31)) return FATHOM_ERR_INVALID_ARG;
+    if (!dims_ok(D, 1)) return FATHOM_ERR_UNSUPPORTED;
+    if (H == 0 || n == 0) return FATHOM_OK;
+    const int64_t nb = ceil_div(n, kBlockTokens);
+    if (nb_stride < nb) return FATHOM_ERR_INVALID_ARG;
+    if (!aligned(planes, 8) || !aligned(store, 16)) return FATHOM_ERR_UNSUPPORTED;
+    FATHOM_TRY(check_device_ptr(planes));
+    FATHOM_TRY(check_device_ptr(store));
+    return launch_tm_from_planes(planes, H, D, n, nb_stride, store, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fathom_nibbles_from_planes(const uint64_t* planes, int64_t H, int D, int64_t n, int64_t nb_stride,

@@ -40,7 +40,7 @@ EXPORTS = (
     "fathom_device_status", "fathom_calibrate_workspace_bytes", "fathom_calibrate",
     "fathom_union_attention_workspace_bytes", "fathom_union_attention",
     "fathom_nibbles_from_planes", "fathom_scan_nibbles", "fathom_layer_budgets_workspace_bytes",
-    "fathom_layer_budgets", "fathom_pack_rotated",
+    "fathom_layer_budgets", "fathom_pack_rotated", "fathom_nibbles_tm_from_planes", "fathom_scan_nibbles_tm",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -85,6 +85,8 @@ def load(path: str | None = None):
         "fathom_scan_topk_noalloc": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, P, P]),
         "fathom_device_status": (I, [I, P]),
         "fathom_pack_rotated": (I, [P, I, I64, I64, I, I64, I64, P, P, P, I64, P]),
+        "fathom_nibbles_tm_from_planes": (I, [P, I64, I, I64, I64, P, P]),
+        "fathom_scan_nibbles_tm": (I, [P, P, I64, I, I64, I64, P, P, P, I, I, P, P, SZ, I, P]),
         "fathom_calibrate_workspace_bytes": (SZ, [I64, I, I]),
         "fathom_calibrate": (I, [P, I, I64, I64, I, I64, I64, P, P, P, P, SZ, P]),
         "fathom_union_attention_workspace_bytes": (SZ, [I64, I, I, I64]),
@@ -238,13 +240,19 @@ def plan_fixed(q: torch.Tensor, r: int, out=None, stream=None, bits: int = 4):
 
 
 def scan(planes, scales, n: int, active, n_active, q, mode: int = SCAN_DENSE, k: int = 0,
-         scores=None, cand=None, stream=None, nibbles: bool = False):
+         scores=None, cand=None, stream=None, nibbles: bool = False, token_major: bool = False):
     """Scores [H][G][n] (DENSE) or the candidate buffer (CANDIDATE).  With
     ``nibbles`` the first argument is the nibble store (every active channel
-    read at 4 bits)."""
+    read at 4 bits); with ``token_major`` it is the token-major store of
+    ``nibbles_tm_from_planes`` (the same scores)."""
     H, G, D = q.shape
-    nbs = planes.shape[-1]
-    fn, name = (lib().fathom_scan_nibbles, "fathom_scan_nibbles") if nibbles else (lib().fathom_scan, "fathom_scan")
+    nbs = scales.shape[-1]
+    if token_major:
+        fn, name = lib().fathom_scan_nibbles_tm, "fathom_scan_nibbles_tm"
+    elif nibbles:
+        fn, name = lib().fathom_scan_nibbles, "fathom_scan_nibbles"
+    else:
+        fn, name = lib().fathom_scan, "fathom_scan"
     if mode == SCAN_DENSE:
         if scores is None:
             scores = torch.empty((H, G, n), dtype=torch.float32, device=q.device)
@@ -266,6 +274,17 @@ def nibbles_from_planes(planes, n: int, out=None, stream=None):
         out = torch.empty_like(planes)
     _check(lib().fathom_nibbles_from_planes(_p(planes), H, D, n, nbs, _p(out), _stream(stream)),
            "fathom_nibbles_from_planes")
+    return out
+
+
+def nibbles_tm_from_planes(planes, n: int, out=None, stream=None):
+    """The token-major 4-bit store uint8 [H][64*nb_stride][D/2] of the codes
+    the planes hold (two channels per byte, channel 2c in the low nibble)."""
+    H, D, _, nbs = planes.shape
+    if out is None:
+        out = torch.zeros((H, 64 * nbs, D // 2), dtype=torch.uint8, device=planes.device)
+    _check(lib().fathom_nibbles_tm_from_planes(_p(planes), H, D, n, nbs, _p(out), _stream(stream)),
+           "fathom_nibbles_tm_from_planes")
     return out
 
 
@@ -392,12 +411,13 @@ class Step:
     candidate pass could not prove its top-k exact.  Buffers are allocated
     once; ``run`` launches only library kernels.  With ``nibbles`` the scans
     read that nibble store (every active channel whole) instead of the
-    planes."""
+    planes; with ``token_major`` too, it is the token-major store."""
 
     def __init__(self, planes, scales, n: int, sigma2, G: int, k: int, budget=48, fixed_r: int | None = None,
-                 fixed_bits: int = 4, nibbles=None):
+                 fixed_bits: int = 4, nibbles=None, token_major: bool = False):
         self.planes, self.scales, self.n, self.sigma2, self.k = planes, scales, n, sigma2, k
         self.nibbles = nibbles
+        self.token_major = token_major   # ``nibbles`` is the token-major store
         self.store = planes if nibbles is None else nibbles
         self.H, self.D = sigma2.shape
         self.G = G
@@ -425,12 +445,12 @@ class Step:
     def run_prepare(self, q):
         _, active, n_active, _ = self.plan_out
         return scan(self.store, self.scales, self.n, active, n_active, q, SCAN_PREPARE, self.k, cand=self.cand,
-                    nibbles=self.nibbles is not None)
+                    nibbles=self.nibbles is not None, token_major=self.token_major)
 
     def run_filter(self, q):
         _, active, n_active, _ = self.plan_out
         return scan(self.store, self.scales, self.n, active, n_active, q, SCAN_FILTER, self.k, cand=self.cand,
-                    nibbles=self.nibbles is not None)
+                    nibbles=self.nibbles is not None, token_major=self.token_major)
 
     def run_scan(self, q):
         self.run_prepare(q)
@@ -459,6 +479,6 @@ class Step:
         for h in bad:
             sl = slice(h, h + 1)
             sc = scan(self.store[sl], self.scales[sl], self.n, active[sl], n_active[sl], q[sl], SCAN_DENSE,
-                      nibbles=self.nibbles is not None)
+                      nibbles=self.nibbles is not None, token_major=self.token_major)
             topk(1, self.G, self.n, self.k, scores=sc, out=(idx[sl], uni[sl], cnt[sl]))
         return len(bad)

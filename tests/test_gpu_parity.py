@@ -603,3 +603,58 @@ def test_pack_rotated_identity_is_pack_and_appends(fathom_gpu):
     assert st == fathom_gpu.OK
     torch.cuda.synchronize()
     assert torch.equal(pa, pb) and torch.equal(sa, sb)
+
+
+# --------------------------------------------------------------------------
+# Token-major 4-bit comparator (byte-accounting section: a serving stack's
+# 4-bit K copy, one row of D/2 bytes per token, read for r chosen channels).
+# --------------------------------------------------------------------------
+def _tm_codes(store: np.ndarray, n: int) -> np.ndarray:
+    """Codes [H][D][n] from the token-major rows (low nibble = even channel)."""
+    lo, hi = store & 15, store >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(store.shape[0], store.shape[1], -1)   # [H][tokens][D]
+    return codes[:, :n].transpose(0, 2, 1)
+
+
+def _cm_codes(nib_words: np.ndarray, n: int) -> np.ndarray:
+    """Codes [H][D][n] from the oracle's channel-major nibble words [H][D][4][nbs]."""
+    H, D, _, nbs = nib_words.shape
+    sh = (np.arange(16, dtype=np.uint64) * np.uint64(4))
+    c = (nib_words[..., None] >> sh) & np.uint64(15)             # [H][D][4 words][nbs][16]
+    c = c.transpose(0, 1, 3, 2, 4).reshape(H, D, nbs * 64)      # token 64b + 16w + e
+    return c[:, :, :n].astype(np.uint8)
+
+
+@pytest.mark.parametrize("w", [
+    dataclasses.replace(inputs.LAYER_32K, name="tm-8x32768", H=8),
+    dataclasses.replace(inputs.TINY, name="tm-g3-d64", H=3, n=5001, D=64, G=3, seed=31),
+    dataclasses.replace(inputs.TINY, name="tm-g8-d256", H=2, n=2500, D=256, G=8, seed=32),
+    dataclasses.replace(inputs.TINY, name="tm-direct", H=2, n=1500, seed=33),
+], ids=lambda w: w.name)
+def test_token_major_store_and_scan(fathom_gpu, orc, w):
+    """The token-major rows hold the oracle's 4-bit codes; the scan over them
+    gives the oracle's full-depth scores of the chosen channels within
+    tolerance and the channel-major nibble scan's to fp32 rounding, and its
+    candidate step picks exactly the top-k of its own dense scores."""
+    k, q, s2 = make(w)
+    planes, scales = fathom_gpu.pack(k)
+    tm = fathom_gpu.nibbles_tm_from_planes(planes, w.n)
+    torch.cuda.synchronize()
+    assert tm.shape == (w.H, 64 * planes.shape[-1], w.D // 2)
+    ref = orc.pack_nibbles(keys_for_oracle(k), nb_stride=planes.shape[-1])
+    assert np.array_equal(_tm_codes(tm.cpu().numpy(), w.n), _cm_codes(ref, w.n))
+    r = min(32, w.D // 4)
+    depth, active, na = fathom_gpu.plan_fixed(q, r)
+    s_tm = fathom_gpu.scan(tm, scales, w.n, active, na, q, token_major=True)
+    nib = fathom_gpu.nibbles_from_planes(planes, w.n)
+    s_cm = fathom_gpu.scan(nib, scales, w.n, active, na, q, nibbles=True)
+    torch.cuda.synchronize()
+    o_scores, o_l1 = orc.scan(np_u64(planes), np_u16(scales), depth.cpu().numpy(), q.cpu().numpy(), w.n)
+    assert_scores_close(s_tm.cpu().numpy(), o_scores, o_l1)
+    assert_scores_close(s_tm.cpu().numpy(), s_cm.cpu().numpy().astype(np.float64), o_l1)
+    st = fathom_gpu.Step(planes, scales, w.n, s2, w.G, w.k, fixed_r=r, nibbles=tm, token_major=True)
+    idx, uni, cnt = st.run(q)
+    d_idx, d_uni, d_cnt = fathom_gpu.topk(w.H, w.G, w.n, w.k, scores=s_tm)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, d_idx) and torch.equal(uni, d_uni) and torch.equal(cnt, d_cnt)
+    assert_topk_sets_match(idx.cpu().numpy(), orc.topk(o_scores, w.k)[0], o_scores, o_l1, w.k)
