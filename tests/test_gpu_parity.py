@@ -445,6 +445,16 @@ def test_union_attention_random_unions(fathom_gpu, orc):
     tol = _attention_tolerance(_as_np(k), _as_np(v), _as_np(q), ref_uni, ref_cnt)
     assert np.all(np.abs(got - ref) <= tol + 1e-30), np.max(np.abs(got - ref) - tol)
     assert not np.any(got[3]) and not np.any(got[4])
+    # Rows 130 floats apart (not 16-byte multiples): the general kernel, same answer.
+    kp = torch.zeros((w.H, w.n, w.D + 2), dtype=k.dtype, device=DEV)
+    vp = torch.zeros_like(kp)
+    kp[:, :, :w.D] = k
+    vp[:, :, :w.D] = v
+    out2 = fathom_gpu.union_attention(kp[:, :, :w.D], vp[:, :, :w.D], q, torch.from_numpy(bad).to(DEV),
+                                      torch.from_numpy(cnt).to(DEV))
+    torch.cuda.synchronize()
+    got2 = out2.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got2 - ref) <= tol + 1e-30), np.max(np.abs(got2 - ref) - tol)
 
 
 def test_union_attention_after_a_step(fathom_gpu, orc):

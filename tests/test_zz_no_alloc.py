@@ -83,6 +83,20 @@ def test_noalloc_takes_no_device_memory_and_checks_outputs_first(fathom_gpu):
     free1 = torch.cuda.mem_get_info()[0]
     assert free0 == free1
     assert torch.all(out[2] >= 0)
+    # The call also captures into a CUDA graph (no allocation, no implicit
+    # synchronisation) and the replay gives the same result.
+    ref = tuple(t.clone() for t in out)
+    for t in out:
+        t.fill_(-7)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side), torch.cuda.graph(graph, stream=side):
+        fathom.scan_topk_noalloc(planes, scales, w.n, active, na, q, w.k, out=out, stream=side)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(out, ref))
+    del graph
     lib = fathom.lib()
     misaligned = ctypes.c_void_p(out[0].data_ptr() + 2)
     st = lib.fathom_scan_topk_noalloc(fathom._p(planes), fathom._p(scales), w.H, w.D, w.n, planes.shape[-1],
