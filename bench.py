@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--host-resident", action="store_true",
                     help="index in page-locked host memory, read over the host link (multi-session case)")
     ap.add_argument("--sessions", type=int, default=3, help="sessions of the host-resident case")
+    ap.add_argument("--case", choices=tuple(CASES), default=None,
+                    help="one small timed case, for profiling a single kernel (see CASES)")
     ap.add_argument("--quiet", action="store_true")
     return ap.parse_args(argv)
 
@@ -905,9 +907,83 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ----------------------------------------------------------------------------
+# Small single-kernel cases (profiling targets; a few GB on the device)
+# ----------------------------------------------------------------------------
+def _case_layer(args, dev):
+    """One layer of the step: 8 groups x 2^20 keys, B = 48 (the chain the
+    layer-sequential step launches 36 times)."""
+    from long_context_decode_bit_b200 import fathom, inputs
+    w = dataclasses.replace(inputs.STEP_1M, H=8)
+    planes, scales, s2, q, _ = build_index(w, dev, log=lambda *a: None)
+    st = fathom.Step(planes, scales, w.n, s2, w.G, w.k, budget=48)
+    return w, (lambda ev: st.run(q, check_overflow=False))
+
+
+def _case_rows(args, dev):
+    """The union's winner rows rebuilt from the planes, 288 groups x 131,072 keys."""
+    import torch
+    from long_context_decode_bit_b200 import fathom, inputs
+    w = inputs.STEP_128K
+    planes, scales, s2, q, _ = build_index(w, dev, log=lambda *a: None)
+    st = fathom.Step(planes, scales, w.n, s2, w.G, w.k, budget=48)
+    st.run(q)
+    _, uni, cnt = st.topk_out
+    out = torch.empty((w.H, uni.shape[1], w.D), dtype=torch.float32, device=dev)
+    return w, (lambda ev: fathom.dequant_rows(planes, scales, w.n, uni, cnt, out=out))
+
+
+def _case_attention(args, dev):
+    """Attention over 2,048 scattered union rows per group, 32 groups of a
+    131,072-key bf16 K/V cache."""
+    import torch
+    from long_context_decode_bit_b200 import fathom, inputs
+    w = dataclasses.replace(inputs.STEP_1M, name="attention-32x131072", H=32, n=131072, seed=inputs.STEP_1M.seed + 7)
+    kc, vc = inputs.keys(w, 0, w.H, device=dev), inputs.values(w, 0, w.H, device=dev)
+    q = inputs.queries(w, 0, w.H, device=dev).float().contiguous()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(97)
+    M = w.G * w.k
+    uni = torch.sort(torch.randperm(w.n, generator=gen, device=dev)[:M].repeat(w.H, 1), dim=1)[0].to(torch.int32)
+    cnt = torch.full((w.H,), M, dtype=torch.int32, device=dev)
+    out = torch.empty((w.H, w.G, w.D), dtype=torch.float32, device=dev)
+    ws = torch.empty(fathom.union_attention_workspace_bytes(w.H, w.G, w.D, M), dtype=torch.uint8, device=dev)
+    return w, (lambda ev: fathom.union_attention(kc, vc, q, uni.contiguous(), cnt, out=out, workspace=ws))
+
+
+def _case_token_major(args, dev):
+    """The fixed 136-bit step over the token-major 4-bit copy, 16 groups x 2^20 keys."""
+    from long_context_decode_bit_b200 import fathom, inputs
+    w = dataclasses.replace(inputs.STEP_1M, H=16)
+    planes, scales, s2, q, _ = build_index(w, dev, log=lambda *a: None)
+    tm = fathom.nibbles_tm_from_planes(planes, w.n)
+    st = fathom.Step(planes, scales, w.n, s2, w.G, w.k, fixed_r=32, nibbles=tm, token_major=True)
+    return w, (lambda ev: st.run(q, check_overflow=False))
+
+
+CASES = {"layer-8x1048576": _case_layer, "rows-288x131072": _case_rows, "attention-32x131072": _case_attention,
+         "token-major-16x1048576": _case_token_major}
+
+
+def run_case(args):
+    import torch
+    from long_context_decode_bit_b200 import fathom
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    fathom.load()
+    w, fn = CASES[args.case](args, dev)
+    fn(None)
+    torch.cuda.synchronize(dev)
+    tot, _ = time_steps(fn, args.steps, args.warmup, dev)
+    return {"case": args.case, "workload": w.name, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_call": tot / args.steps}
+
+
 def main(argv=None):
     args = parse_args(argv)
-    if args.impl == "reference":
+    if args.case is not None:
+        res = run_case(args)
+    elif args.impl == "reference":
         res = run_reference(args)
     elif args.host_resident:
         res = run_host_resident(args)
