@@ -44,8 +44,8 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("fathom", "reference"), default="fathom")
     ap.add_argument("--workload", default="qwen3-8b-step-288x1048576")
     ap.add_argument("--budget", type=int, default=48)
@@ -100,7 +100,7 @@ def barrier(device=None):
 # clocks, peaks, profile-derived traffic
 # ----------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi samples (200 ms) while the timed region runs."""
+    """nvidia-smi samples (every 50 ms) while the timed region runs."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -114,7 +114,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except (OSError, FileNotFoundError):
@@ -779,8 +779,8 @@ def host_resident_entry(w, planes, scales, sigma2, q, k, device, log):
         fb = st.repair(q)
         alg = plan_bytes(st, w)[0]
         with ClockSampler(gpu_id) as clk:
-            tot, _ = time_steps(one, 3, 1, device)
-        ms = tot / 3
+            tot, _ = time_steps(one, 6, 1, device)
+        ms = tot / 6
         out[bname] = {"ms_per_step": ms, "keys_per_s": w.H * w.n / (ms / 1e3), "alg_bytes": alg,
                       "read_bits_per_token": alg * 8 / (w.H * w.n), "link_GBps": alg / (ms / 1e3) / 1e9,
                       "link_frac": alg / (ms / 1e3) / 1e9 / link, "fallback_groups": fb, "clocks": clk.summary()}

@@ -244,6 +244,10 @@ __device__ __forceinline__ void depth_class(uint32_t& wrow, uint32_t& cf, int co
                                             float2 (&acc)[8][head_pairs<G>()])
 {
     constexpr uint32_t kCf = kBlocksPerWarp * coef_pairs<G>() * 8;
+    // Two channels per iteration (fewer loop and address instructions:
+    // 2.96 -> 2.90 ms at 288 x 1M, G = 4); G >= 5 keeps one, as two would spill.
+    constexpr int kUnroll = G <= 4 ? 2 : 1;
+#pragma unroll kUnroll
     for (int i = 0; i < count; ++i) {
         float v[8];
         channel_values<T, NIB>(wrow, l, v);
