@@ -45,7 +45,31 @@ __device__ __forceinline__ float load_key<__nv_bfloat16>(const __nv_bfloat16* p)
     return __bfloat162float(__ldg(p));
 }
 
+// 16 bytes of keys (8 bf16 or 4 fp32 channels) as floats.
 template <typename T>
+__device__ __forceinline__ void load16(const T* p, float (&x)[16 / sizeof(T)]);
+
+template <>
+__device__ __forceinline__ void load16<float>(const float* p, float (&x)[4])
+{
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+
+template <>
+__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8])
+{
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+
+template <typename T, bool VEC>
 __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const T* __restrict__ keys, int64_t H, int64_t n, int D, int64_t stride_h,
             int64_t stride_tok, uint64_t* __restrict__ planes, uint16_t* __restrict__ scales,
@@ -60,12 +84,38 @@ pack_kernel(const T* __restrict__ keys, int64_t H, int64_t n, int D, int64_t str
     const int64_t t0 = b0 * kBlockTokens;
     const int tid = threadIdx.x;
 
-    // Stage keys: each warp reads one token row of 32 channels per step.
+    // Stage keys.  VEC (16-byte aligned rows): each thread reads 16-byte
+    // pieces of token rows, all of its reads issued before the stores;
+    // otherwise one element per read, a warp per token row.
     const T* kg = keys + h * stride_h + c0;
-    for (int idx = tid; idx < kPackTokens * kPackCh; idx += kPackThreads) {
-        const int tok = idx / kPackCh, ch = idx % kPackCh;
-        const int64_t i = t0 + tok;
-        tile[tok][ch] = (i < n) ? load_key(kg + i * stride_tok + ch) : 0.0f;
+    if (VEC) {
+        constexpr int E = 16 / sizeof(T);                 // channels per piece
+        constexpr int kPieces = kPackTokens * kPackCh / E;
+        constexpr int kPer = kPieces / kPackThreads;
+        float x[kPer][E];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int idx = tid + u * kPackThreads;
+            const int tok = idx / (kPackCh / E), q = idx % (kPackCh / E);
+            const int64_t i = t0 + tok;
+            if (i < n) load16<T>(kg + i * stride_tok + q * E, x[u]);
+            else
+#pragma unroll
+                for (int e = 0; e < E; ++e) x[u][e] = 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int idx = tid + u * kPackThreads;
+            const int tok = idx / (kPackCh / E), q = idx % (kPackCh / E);
+#pragma unroll
+            for (int e = 0; e < E; ++e) tile[tok][q * E + e] = x[u][e];
+        }
+    } else {
+        for (int idx = tid; idx < kPackTokens * kPackCh; idx += kPackThreads) {
+            const int tok = idx / kPackCh, ch = idx % kPackCh;
+            const int64_t i = t0 + tok;
+            tile[tok][ch] = (i < n) ? load_key(kg + i * stride_tok + ch) : 0.0f;
+        }
     }
     __syncthreads();
 
@@ -271,13 +321,18 @@ int launch_pack(const void* keys, int key_dtype, int64_t H, int64_t n, int D, in
     const int64_t nb = ceil_div(n, kBlockTokens);
     const dim3 grid(static_cast<unsigned>(ceil_div(nb, kPackBlocks)),
                     static_cast<unsigned>(H * (D / kPackCh)));
-    if (key_dtype == FATHOM_KEYS_F32)
-        pack_kernel<float><<<grid, kPackThreads, 0, stream>>>(
-            static_cast<const float*>(keys), H, n, D, stride_h, stride_tok, planes, scales, nb_stride, nb);
-    else
-        pack_kernel<__nv_bfloat16><<<grid, kPackThreads, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(keys), H, n, D, stride_h, stride_tok, planes, scales,
-            nb_stride, nb);
+    const int64_t esz = key_dtype == FATHOM_KEYS_F32 ? 4 : 2;
+    const bool vec = (reinterpret_cast<uintptr_t>(keys) & 15) == 0 && (stride_tok * esz) % 16 == 0 &&
+                     (stride_h * esz) % 16 == 0;
+    if (key_dtype == FATHOM_KEYS_F32) {
+        const float* k = static_cast<const float*>(keys);
+        if (vec) pack_kernel<float, true><<<grid, kPackThreads, 0, stream>>>(k, H, n, D, stride_h, stride_tok, planes, scales, nb_stride, nb);
+        else pack_kernel<float, false><<<grid, kPackThreads, 0, stream>>>(k, H, n, D, stride_h, stride_tok, planes, scales, nb_stride, nb);
+    } else {
+        const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(keys);
+        if (vec) pack_kernel<__nv_bfloat16, true><<<grid, kPackThreads, 0, stream>>>(k, H, n, D, stride_h, stride_tok, planes, scales, nb_stride, nb);
+        else pack_kernel<__nv_bfloat16, false><<<grid, kPackThreads, 0, stream>>>(k, H, n, D, stride_h, stride_tok, planes, scales, nb_stride, nb);
+    }
     return launch_status();
 }
 

@@ -668,3 +668,17 @@ def test_token_major_store_and_scan(fathom_gpu, orc, w):
     torch.cuda.synchronize()
     assert torch.equal(idx, d_idx) and torch.equal(uni, d_uni) and torch.equal(cnt, d_cnt)
     assert_topk_sets_match(idx.cpu().numpy(), orc.topk(o_scores, w.k)[0], o_scores, o_l1, w.k)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_pack_of_unaligned_rows_equals_contiguous(fathom_gpu, dtype):
+    """Key rows 130 elements apart (not 16-byte multiples) take the element-wise
+    staging; the index equals that of the same keys stored contiguously."""
+    w = dataclasses.replace(inputs.LAYER_32K, name="pack-unaligned", H=2, n=3001, seed=79)
+    k = inputs.keys(w, 0, w.H, device=DEV).to(dtype).contiguous()
+    kp = torch.zeros((w.H, w.n, w.D + 2), dtype=dtype, device=DEV)
+    kp[:, :, :w.D] = k
+    p0, s0 = fathom_gpu.pack(k)
+    p1, s1 = fathom_gpu.pack(kp[:, :, :w.D])
+    torch.cuda.synchronize()
+    assert torch.equal(p0, p1) and torch.equal(s0, s1)
