@@ -52,6 +52,7 @@ typedef struct CUstream_st* fathom_stream_t; /* same type as cudaStream_t */
 #define FATHOM_ERR_WORKSPACE (-4)   /* caller buffer smaller than the *_bytes() query */
 #define FATHOM_ERR_TIMEOUT (-5)     /* a bounded device wait gave up; see fathom_device_status() */
 #define FATHOM_ERR_OVERFLOW (-6)    /* candidate pass could not prove its top-k exact */
+#define FATHOM_ERR_BOUNDS (-7)      /* debug build only: a device-side bounds check failed (the access was skipped) */
 
 /* Key element types for fathom_pack. */
 #define FATHOM_KEYS_F32 0
@@ -410,7 +411,8 @@ size_t fathom_topk_workspace_bytes(int64_t H, int G, int64_t n, int k);
  *              group's idx and union_idx are unspecified and the caller
  *              reruns it with a DENSE scan; FATHOM_ERR_TIMEOUT for every
  *              group while the device fault word is set (a scan's bounded
- *              wait gave up: nothing of that step is valid).
+ *              wait gave up: nothing of that step is valid), or
+ *              FATHOM_ERR_BOUNDS in a debug build whose bounds check failed.
  *   workspace, ws_bytes  DEVICE scratch of fathom_topk_workspace_bytes()
  *              bytes (may be NULL when that is 0).
  */
@@ -516,8 +518,10 @@ int fathom_scan_topk_noalloc(const uint64_t* planes, const uint16_t* scales, int
 /*
  * fathom_device_status -- FATHOM_ERR_TIMEOUT if a kernel of this library on
  * the current device has given up a bounded wait since the word was last
- * cleared, else FATHOM_OK (or FATHOM_ERR_CUDA).  (The paper has no
- * counterpart: this is the library's own failure report.)
+ * cleared; else FATHOM_ERR_BOUNDS if, in a build with device-side bounds
+ * checks (FATHOM_DEBUG_BOUNDS), a check failed and its access was skipped;
+ * else FATHOM_OK (or FATHOM_ERR_CUDA).  (The paper has no counterpart: this
+ * is the library's own failure report.)
  *
  * Reads the device's fault word in stream order and synchronises `stream`;
  * with clear != 0 a set word is reset to 0 afterwards.  The word is one per

@@ -3,10 +3,13 @@
 ``python -m long_context_decode_bit_b200.build [--force] [--ptxas-v] [--test-hooks]``
 
 ``--test-hooks`` builds ``libfathom_testhooks.so`` instead: the same sources
-with a short ring-wait poll limit and a switch (the environment variable
-``FATHOM_TEST_WITHHOLD_ARRIVAL=1``) that makes the scan withhold one ring
-arrival, so that a test can watch a bounded wait run out and the error
-reach the host.  The product never loads it.
+with a short ring-wait poll limit, the device-side bounds checks of
+``FATHOM_DEBUG_BOUNDS`` (a failed check sets the fault word's bounds bit and
+skips the access; ``fathom_device_status`` then returns FATHOM_ERR_BOUNDS),
+and two switches for tests: ``FATHOM_TEST_WITHHOLD_ARRIVAL=1`` makes the
+scan withhold one ring arrival (a bounded wait runs out), and
+``FATHOM_TEST_SHRINK_CAP=1`` makes the checks allow only half of the
+candidate entries (a check fails).  The product never loads it.
 """
 from __future__ import annotations
 
@@ -23,7 +26,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfathom.so")
 TEST_LIB = os.path.join(PKG, "libfathom_testhooks.so")
 # about 65k polls of at most ~1 us each: tens of ms, far above any normal wait
-TEST_DEFINES = ["-DFATHOM_TEST_HOOKS", "-DFATHOM_SPIN_LIMIT=65536"]
+TEST_DEFINES = ["-DFATHOM_TEST_HOOKS", "-DFATHOM_SPIN_LIMIT=65536", "-DFATHOM_DEBUG_BOUNDS"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

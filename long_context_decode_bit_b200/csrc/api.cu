@@ -205,6 +205,7 @@ const char* fathom_status_string(int status)
         case FATHOM_ERR_WORKSPACE: return "buffer too small";
         case FATHOM_ERR_TIMEOUT: return "device wait timed out";
         case FATHOM_ERR_OVERFLOW: return "candidate pass could not prove the top-k exact";
+        case FATHOM_ERR_BOUNDS: return "device bounds check failed (debug build)";
         default: return "unknown status";
     }
 }

@@ -55,6 +55,26 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
     return cuda_status(cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...));
 }
 
+// Device fault word bits: 1 = a bounded wait gave up; 2 = a bounds check of
+// the debug build failed.
+constexpr int32_t kFaultTimeout = 1;
+constexpr int32_t kFaultBounds = 2;
+
+// Debug build (FATHOM_DEBUG_BOUNDS): `ok` guards a memory access; a false
+// check sets the fault word's bounds bit and the caller skips the access.
+// Release builds compile the check away.
+__device__ __forceinline__ bool bounds_ok(bool ok, int32_t* fault)
+{
+#ifdef FATHOM_DEBUG_BOUNDS
+    if (!ok) atomicOr(fault, kFaultBounds);
+    return ok;
+#else
+    (void)ok;
+    (void)fault;
+    return true;
+#endif
+}
+
 // SM count of the current device (queried once per device; launch.cu).
 int device_sm_count(int* sms);
 

@@ -1,4 +1,5 @@
-// Device fault word: set by a kernel whose bounded wait gave up.
+// Device fault word: set by a kernel whose bounded wait gave up (bit 0), or,
+// in the debug build, whose bounds check failed (bit 1).
 //
 // The scan's shared-memory ring waits on mbarriers with a poll limit.  A wait
 // that runs out (which a correct launch never does) makes the kernel set
@@ -60,5 +61,5 @@ extern "C" int fathom_device_status(int clear, fathom_stream_t stream)
         if (e == cudaSuccess) e = cudaStreamSynchronize(s);
         if (e != cudaSuccess) return cuda_status(e);
     }
-    return v ? FATHOM_ERR_TIMEOUT : FATHOM_OK;
+    return (v & kFaultTimeout) ? FATHOM_ERR_TIMEOUT : ((v & kFaultBounds) ? FATHOM_ERR_BOUNDS : FATHOM_OK);
 }

@@ -91,6 +91,7 @@ struct ScanArgs {
     int tiles_per_cta;
     int mode;
     int32_t* fault;            // device fault word: set when a ring wait ran out
+    int64_t cap_check;         // entries per head the bounds checks allow (cap; less only in a test build)
     bool nib;                  // `planes` is the nibble store, read at 4 bits
 #ifdef FATHOM_TEST_HOOKS
     bool withhold;             // test build: withhold one ring arrival (see the producer)
@@ -402,8 +403,9 @@ scan_kernel(const ScanArgs a)
                 const int64_t row = (h * D + (src_rc >> 2)) * kPlanes + (src_rc & 3);
                 const int64_t vb = valid_blocks - 2 * part;
                 const int bytes = vb >= 2 ? 16 : (vb == 1 ? 8 : 0);
-                const uint64_t* src = a.planes + row * a.nb_stride + (bytes ? b0 + 2 * part : 0);
-                cp_async16(&S.words[st][r * kScanTileBlocks + 2 * part], src, bytes);
+                const int64_t col = bytes ? b0 + 2 * part : 0;
+                if (bounds_ok(row < static_cast<int64_t>(gridDim.y) * D * kPlanes && col + 2 <= a.nb_stride, a.fault))
+                    cp_async16(&S.words[st][r * kScanTileBlocks + 2 * part], a.planes + row * a.nb_stride + col, bytes);
             }
             // Scale rows: pieces of 16 B (8 blocks each), kScanTileBlocks / 8 per channel.
             constexpr int kScalePieces = kScanTileBlocks / 8;
@@ -412,8 +414,10 @@ scan_kernel(const ScanArgs a)
                 const int j = S.chan[c0 + c] & 0xFF;
                 const int64_t vb = valid_blocks - 8 * part;
                 const int bytes = vb >= 8 ? 16 : (vb > 0 ? static_cast<int>(vb) * 2 : 0);
-                const uint16_t* src = a.scales + (h * D + j) * a.nb_stride + (bytes ? b0 + 8 * part : 0);
-                cp_async16(&S.rawscale[st][c * kScanTileBlocks + 8 * part], src, bytes);
+                const int64_t col = bytes ? b0 + 8 * part : 0;
+                if (bounds_ok(j < D && col + 8 <= a.nb_stride, a.fault))
+                    cp_async16(&S.rawscale[st][c * kScanTileBlocks + 8 * part], a.scales + (h * D + j) * a.nb_stride + col,
+                               bytes);
             }
 #ifdef FATHOM_TEST_HOOKS
             // Test build only: lane 0 of the first CTA of head 0 withholds its
@@ -495,7 +499,8 @@ scan_kernel(const ScanArgs a)
                     const bool in = tok0 + off < a.n;
 #pragma unroll
                     for (int g = 0; g < G; ++g)
-                        a.sample[(h * G + g) * a.n_sample + lt0 + off] = in ? acc_at<G>(acc, m, g) : -INFINITY;
+                        if (bounds_ok(lt0 + off < a.n_sample, a.fault))
+                            a.sample[(h * G + g) * a.n_sample + lt0 + off] = in ? acc_at<G>(acc, m, g) : -INFINITY;
                 }
             } else {
                 const int64_t ptile = ltile * a.tile_stride;
@@ -506,10 +511,11 @@ scan_kernel(const ScanArgs a)
                     if (!whole && i >= a.n) return;
                     const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
                     if (S.direct[g]) {
-                        ent_h[g * a.cap + i] = ent;
+                        if (bounds_ok(i < a.cap_check, a.fault)) ent_h[g * a.cap + i] = ent;
                     } else {
                         const int p = atomicAdd(&S.tile_cnt[ti][g], 1);
-                        if (p < a.tslot) ent_h[g * a.cap + ptile * a.tslot + p] = ent;
+                        if (p < a.tslot && bounds_ok(ptile * a.tslot + p < a.cap_check, a.fault))
+                            ent_h[g * a.cap + ptile * a.tslot + p] = ent;
                     }
                 };
                 // Survivor mask over (head, token): one compare per score and
@@ -686,6 +692,15 @@ int launch_scan(const uint64_t* planes, const uint16_t* scales, int64_t H, int D
     a.tile_counts = reinterpret_cast<int32_t*>(base + L.off_counts);
     a.entries = reinterpret_cast<int2*>(base + L.off_entries);
     a.cap = L.cap;
+    a.cap_check = L.cap;
+#ifdef FATHOM_TEST_HOOKS
+    {
+        // Test build only: let the bounds checks allow half the entries, so
+        // that a test sees a failed check reach the host as FATHOM_ERR_BOUNDS.
+        const char* e = getenv("FATHOM_TEST_SHRINK_CAP");
+        if (e != nullptr && e[0] == '1') a.cap_check = L.cap / 2;
+    }
+#endif
     a.tslot = L.tslot;
     a.n_sample = L.n_sample;
     if (mode == FATHOM_SCAN_CANDIDATE || mode == FATHOM_SCAN_PREPARE) {

@@ -57,6 +57,7 @@ struct TmArgs {
     int64_t cap, tslot, n_sample, tile_stride, tiles;
     int tiles_per_cta;
     int mode;
+    int32_t* fault;            // device fault word (bounds bit of the debug build)
 };
 
 template <int G>
@@ -165,7 +166,7 @@ scan_tm_kernel(const TmArgs a)
             const int64_t b0u = (static_cast<int64_t>(blockIdx.x) * a.tiles_per_cta + u / kTmBlocksPerWarp) *
                                 a.tile_stride * kScanTileBlocks;
             const int bl = warp * kTmBlocksPerWarp + u % kTmBlocksPerWarp;
-            if (bl < a.nb - b0u) {
+            if (bl < a.nb - b0u && bounds_ok(b0u + bl < a.nb_stride, a.fault)) {
                 const unsigned char* src = st_h + (b0u + bl) * kBlockTokens * rowb;
                 unsigned char* dst = mybuf + (u & 1) * kBlockTokens * pitch;
                 for (int e = lane; e < kBlockTokens * cpr; e += 32) {
@@ -278,10 +279,11 @@ scan_tm_kernel(const TmArgs a)
                     const float sv = acc_g(m, g);
                     const int2 ent = make_int2(static_cast<int>(i), __float_as_int(sv));
                     if (S.direct[g]) {
-                        ent_h[g * a.cap + i] = ent;
+                        if (bounds_ok(i < a.cap, a.fault)) ent_h[g * a.cap + i] = ent;
                     } else if (!(sv < S.tau[g])) {   // a NaN score counts as reaching tau
                         const int p = atomicAdd(&S.tile_cnt[ti][g], 1);
-                        if (p < a.tslot) ent_h[g * a.cap + ptile * a.tslot + p] = ent;
+                        if (p < a.tslot && bounds_ok(ptile * a.tslot + p < a.cap, a.fault))
+                            ent_h[g * a.cap + ptile * a.tslot + p] = ent;
                     }
                 }
             }
@@ -382,6 +384,10 @@ int launch_scan_tm(const uint8_t* store, const uint16_t* scales, int64_t H, int 
                    void* cand, int k, cudaStream_t stream)
 {
     TmArgs a{};
+    {
+        const int st = device_fault_word(&a.fault);
+        if (st) return st;
+    }
     a.store = store;
     a.scales = scales;
     a.nb_stride = nb_stride;

@@ -191,7 +191,9 @@ __device__ bool load_lists(const TopkArgs& a, int64_t h, int32_t* lists, int* fa
     const int32_t faulted = __ldcg(a.fault);   // a scan whose ring wait gave up left void scores
     if (*failed || faulted) {
         for (int i = threadIdx.x; i < gk; i += blockDim.x) a.union_idx[h * gk + i] = -1;
-        if (threadIdx.x == 0) a.union_count[h] = faulted ? FATHOM_ERR_TIMEOUT : FATHOM_ERR_OVERFLOW;
+        if (threadIdx.x == 0)
+            a.union_count[h] = (faulted & kFaultTimeout) ? FATHOM_ERR_TIMEOUT
+                               : (faulted ? FATHOM_ERR_BOUNDS : FATHOM_ERR_OVERFLOW);
         return false;
     }
     return true;
@@ -257,6 +259,7 @@ __device__ void topk_head(const TopkArgs& a, unsigned char* smem)
             if (c == 0) continue;
             if (base + c > a.gather_cap) { g_bad = 1; continue; }
             const int2* sp = src + t * a.tslot;
+            if (!bounds_ok((t + 1) * a.tslot <= a.cap, const_cast<int32_t*>(a.fault))) continue;
             for (int e0 = 0; e0 < c; e0 += 4) {
                 int2 x[4];
 #pragma unroll

@@ -24,6 +24,7 @@ ERR_CUDA = -3
 ERR_WORKSPACE = -4
 ERR_TIMEOUT = -5
 ERR_OVERFLOW = -6
+ERR_BOUNDS = -7   # debug build: a device-side bounds check failed
 
 KEYS_F32 = 0
 KEYS_BF16 = 1
@@ -400,7 +401,7 @@ def device_status(clear: bool = False, stream=None) -> int:
     a bounded wait since the fault word was last cleared (synchronises the
     stream)."""
     st = int(lib().fathom_device_status(1 if clear else 0, _stream(stream)))
-    if st not in (OK, ERR_TIMEOUT):
+    if st not in (OK, ERR_TIMEOUT, ERR_BOUNDS):
         _check(st, "fathom_device_status")
     return st
 
@@ -473,8 +474,8 @@ class Step:
         bad = torch.nonzero(cnt < 0).flatten().tolist()
         if not bad:
             return 0
-        if int(cnt[bad[0]]) == ERR_TIMEOUT:
-            raise FathomError(ERR_TIMEOUT, "candidate scan (device fault word set)")
+        if int(cnt[bad[0]]) in (ERR_TIMEOUT, ERR_BOUNDS):
+            raise FathomError(int(cnt[bad[0]]), "candidate scan (device fault word set)")
         _, active, n_active, _ = self.plan_out
         for h in bad:
             sl = slice(h, h + 1)
