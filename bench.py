@@ -966,7 +966,21 @@ def _case_token_major(args, dev):
     return w, (lambda ev: st.run(q, check_overflow=False))
 
 
-CASES = {"layer-8x1048576": _case_layer, "rows-288x131072": _case_rows, "attention-32x131072": _case_attention,
+def _case_pack_rotated(args, dev):
+    """Keys rotated inside the pack kernel: 8 Llama-shaped groups x 2^20 bf16 keys."""
+    import torch
+    from long_context_decode_bit_b200 import basis, fathom, inputs
+    w = dataclasses.replace(inputs.STEP_1M_LLAMA, H=8)
+    keys = inputs.keys(w, 0, w.H, device=dev)
+    q = inputs.queries(w, 0, w.H, device=dev).float().contiguous()
+    U = basis.klt_basis(keys[:, :w.n_cal], q).contiguous()
+    nbs = fathom.nb_stride(w.n)
+    planes = torch.zeros((w.H, w.D, 4, nbs), dtype=torch.int64, device=dev)
+    scales = torch.zeros((w.H, w.D, nbs), dtype=torch.int16, device=dev)
+    return w, (lambda ev: fathom.pack_rotated(keys, U, planes=planes, scales=scales))
+
+
+CASES = {"pack-rotated-8x1048576": _case_pack_rotated, "layer-8x1048576": _case_layer, "rows-288x131072": _case_rows, "attention-32x131072": _case_attention,
          "token-major-16x1048576": _case_token_major}
 
 

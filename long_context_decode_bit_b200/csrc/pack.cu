@@ -216,21 +216,28 @@ pack_rotated_kernel(const T* __restrict__ keys, int64_t n, int D, int64_t stride
         }
         __syncthreads();
 
-        float acc[TOK];
+        // Packed fp32x2 FMAs over token pairs: each half is one IEEE fused
+        // multiply-add, so every coordinate still follows the stated chain.
+        float2 acc2[TOK / 2];
 #pragma unroll
-        for (int t = 0; t < TOK; ++t) acc[t] = 0.0f;
+        for (int t = 0; t < TOK / 2; ++t) acc2[t] = make_float2(0.0f, 0.0f);
 #pragma unroll 2
         for (int d = 0; d < D; ++d) {
             const float u = Us[d * C + cl];
+            const float2 uu = make_float2(u, u);
             const float4* xr = reinterpret_cast<const float4*>(Xs + d * kRotRow + tok0);
 #pragma unroll
             for (int v = 0; v < TOK / 4; ++v) {
                 const float4 x = xr[v];
-                acc[4 * v + 0] = fmaf(x.x, u, acc[4 * v + 0]);
-                acc[4 * v + 1] = fmaf(x.y, u, acc[4 * v + 1]);
-                acc[4 * v + 2] = fmaf(x.z, u, acc[4 * v + 2]);
-                acc[4 * v + 3] = fmaf(x.w, u, acc[4 * v + 3]);
+                acc2[2 * v] = __ffma2_rn(make_float2(x.x, x.y), uu, acc2[2 * v]);
+                acc2[2 * v + 1] = __ffma2_rn(make_float2(x.z, x.w), uu, acc2[2 * v + 1]);
             }
+        }
+        float acc[TOK];
+#pragma unroll
+        for (int t = 0; t < TOK / 2; ++t) {
+            acc[2 * t] = acc2[t].x;
+            acc[2 * t + 1] = acc2[t].y;
         }
 
         // Block maximum over the valid tokens, across the lanes of this coordinate.
