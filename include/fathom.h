@@ -20,7 +20,12 @@
  *     address space.  Pointers marked HOST are ordinary host memory.
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream) on the current device.  Outputs are valid
- *     once the stream reaches the call.
+ *     once the stream reaches the call.  The decode-step kernels (plan, scans,
+ *     threshold, top-k, union) are launched with programmatic dependent
+ *     launch: each waits for the previous kernel in the stream to complete
+ *     before it reads anything, so ordering is that of plain launches (also
+ *     under CUDA graph capture), while the next kernel's launch overlaps the
+ *     current one's tail.
  *   - Arguments are validated on the host before anything is launched; a
  *     rejected call launches nothing and returns a negative status.
  *   - A "group" is one KV head of one layer (its G query heads share one
