@@ -104,3 +104,51 @@ def test_step_128k_sampled_groups(orc):
         r_idx = orc.topk(ref, w.k)[0]
         assert_topk_sets_match(idx[h:h + 1].cpu().numpy(), r_idx, ref, l1, w.k)
         assert int(cnt[h]) > 0
+
+
+def test_rotated_llama_step_full_size_sampled(orc):
+    """The rotated Llama-shaped step at its full size (256 groups x 2^20 keys,
+    keys rotated inside the pack kernel): the planes and scales of sampled
+    groups' first 65,536 keys are bit-exact against the oracle's fp32 FMA
+    chain and pack, and the candidate step proves every group exact."""
+    from long_context_decode_bit_b200 import basis
+    w = inputs.STEP_1M_LLAMA
+    dev = torch.device("cuda", 0)
+    planes, scales, s2, q, _ = bench.build_index(w, dev, rotated=True, log=lambda *a: None)
+    st = fathom.Step(planes, scales, w.n, s2, w.G, w.k, budget=48)
+    idx, uni, cnt = st.run(q, check_overflow=False)
+    torch.cuda.synchronize()
+    assert int(torch.min(cnt)) > 0
+    m = 65536
+    for h in (0, 100, 255):
+        # The basis exactly as the index build formed it: per chunk of 8 groups.
+        h0 = h - h % 8
+        kc = inputs.keys(w, h0, min(w.H, h0 + 8), device="cuda")
+        qc = inputs.queries(w, h0, min(w.H, h0 + 8), device="cuda").float().contiguous()
+        U = basis.klt_basis(kc[:, :w.n_cal], qc)[h - h0:h - h0 + 1].contiguous()
+        k = kc[h - h0:h - h0 + 1]
+        del kc
+        p_ref, s_ref = orc.pack_rotated(keys_for_oracle(k[:, :m]), U.cpu().numpy())
+        nb = m // 64
+        assert np.array_equal(np_u64(planes[h:h + 1])[..., :nb], p_ref[..., :nb])
+        assert np.array_equal(np_u16(scales[h:h + 1])[..., :nb], s_ref[..., :nb])
+    del planes, scales
+    torch.cuda.empty_cache()
+
+
+def test_token_major_store_full_size_sampled(step_1m, orc):
+    """The token-major 4-bit copy of the 288 x 2^20 index holds the oracle's
+    codes for sampled groups (every token)."""
+    w, planes, scales, s2, q, st = step_1m
+    for h in (3, 200):
+        tm = fathom.nibbles_tm_from_planes(planes[h:h + 1], w.n)
+        k = inputs.keys(w, h, h + 1, device="cuda")
+        ref = orc.pack_nibbles(keys_for_oracle(k), nb_stride=planes.shape[-1])
+        del k
+        got = tm.cpu().numpy()[:, :w.n]
+        lo, hi = got & 15, got >> 4
+        codes = np.stack([lo, hi], axis=-1).reshape(1, w.n, w.D).transpose(0, 2, 1)
+        sh = np.arange(16, dtype=np.uint64) * np.uint64(4)
+        c = ((ref[..., None] >> sh) & np.uint64(15)).transpose(0, 1, 3, 2, 4).reshape(1, w.D, -1)[:, :, :w.n]
+        assert np.array_equal(codes, c.astype(np.uint8))
+        del tm
