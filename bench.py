@@ -877,6 +877,15 @@ def cpu_baseline(w, k, B, groups, device, log):
                        f"{groups} group(s) on one core")}
 
 
+def reference_keys(n: int, steps: int, warmup: int, groups: int, budget_s: float = 120.0,
+                   keys_per_s: float = 0.6e6) -> int:
+    """Keys per group of one reference-arm step: all n, or a prefix (whole
+    2,048-key tiles, at least 8 of them) small enough that steps + warmup
+    steps of the single-core oracle (about 0.6 M keys/s) take about budget_s."""
+    n_s = int(budget_s * keys_per_s / max(1, steps + warmup) / max(1, groups)) // 2048 * 2048
+    return max(min(n, n_s), min(n, 8 * 2048))
+
+
 def run_reference(args):
     import torch
     rank, world, _ = dist_env()
@@ -888,10 +897,7 @@ def run_reference(args):
         base = dataclasses.replace(base, k=args.k)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     groups = max(1, args.cpu_groups)
-    # Bound the whole run to about two minutes: the oracle scans about 0.6 M
-    # keys/s on one core, so a step takes the first n_s keys of its groups.
-    n_s = int(120 * 0.6e6 / max(1, args.steps + args.warmup) / groups) // 2048 * 2048
-    n_s = max(min(base.n, n_s), min(base.n, 8 * 2048))
+    n_s = reference_keys(base.n, args.steps, args.warmup, groups)
     wl = dataclasses.replace(base, n=n_s) if n_s < base.n else base
     planes, scales, s2, qn = _oracle_sample(wl, groups, dev)
     for _ in range(args.warmup):
