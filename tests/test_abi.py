@@ -142,3 +142,24 @@ def test_missing_library_fails_loudly(tmp_path):
             fathom.load(str(tmp_path / "nope.so"))
     finally:
         fathom._lib = saved
+
+
+def test_step_repair_raises_on_device_fault_statuses(lib):
+    """Step.repair's host decision (no GPU): a TIMEOUT or BOUNDS status in
+    union_count raises instead of starting a dense rerun, and a step whose
+    groups all proved exact needs no repair."""
+    import torch
+    H, D, G, n, k = 3, 128, 4, 4096, 64
+    planes = torch.zeros((H, D, 4, fathom.nb_stride(n)), dtype=torch.int64)
+    scales = torch.zeros((H, D, fathom.nb_stride(n)), dtype=torch.int16)
+    sigma2 = torch.ones((H, D))
+    st = fathom.Step(planes, scales, n, sigma2, G, k)
+    q = torch.zeros((H, G, D))
+    st.topk_out[2].copy_(torch.tensor([5, 7, 9], dtype=torch.int32))
+    assert st.repair(q) == 0
+    for status in (fathom.ERR_TIMEOUT, fathom.ERR_BOUNDS):
+        st.topk_out[2].copy_(torch.tensor([status] * H, dtype=torch.int32))
+        with pytest.raises(fathom.FathomError) as e:
+            st.repair(q)
+        assert e.value.status == status
+    assert lib.fathom_status_string(fathom.ERR_BOUNDS).decode() != "unknown status"
