@@ -125,6 +125,19 @@ def test_rejections_before_any_cuda_call(lib):
     assert lib.fathom_layer_budgets(n, n, 10, 4, 128, 0, 100, n, n, 0, n) == fathom.ERR_INVALID_ARG   # no layer
     assert lib.fathom_layer_budgets(n, n, 10, 4, 100, 5, 100, n, n, 0, n) == fathom.ERR_UNSUPPORTED
     assert lib.fathom_layer_budgets(fake, fake, 10, 4, 128, 5, 100, fake, fake, 64, n) == fathom.ERR_WORKSPACE
+    # keys rotated inside pack: the checks of fathom_pack, plus U's alignment
+    assert lib.fathom_pack_rotated(n, 0, 1, 64, 48, 64 * 48, 48, n, n, n, 16, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_pack_rotated(n, 7, 1, 64, 128, 64 * 128, 128, n, n, n, 16, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_pack_rotated(n, 0, 0, 64, 128, 0, 128, n, n, n, 16, n) == fathom.OK      # nothing to do
+    assert lib.fathom_pack_rotated(n, 0, 1, 1000, 128, 1000 * 128, 128, n, n, n, 15, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_pack_rotated(fake, 0, 1, 64, 128, 64 * 128, 128, ctypes.c_void_p(258), fake, fake, 16,
+                                   n) == fathom.ERR_UNSUPPORTED                                 # U misaligned
+    # the token-major comparator: the checks of fathom_scan and of the nibble store
+    assert lib.fathom_scan_nibbles_tm(n, n, 1, 128, 100, 2, n, n, n, 4, 5, n, n, 0, 1, n) == fathom.ERR_INVALID_ARG
+    assert lib.fathom_scan_nibbles_tm(n, n, 1, 100, 100, 2, n, n, n, 4, 0, n, n, 0, 1, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_nibbles_tm_from_planes(n, 1, 48, 100, 2, n, n) == fathom.ERR_UNSUPPORTED
+    assert lib.fathom_nibbles_tm_from_planes(n, 1, 128, 1000, 15, n, n) == fathom.ERR_INVALID_ARG   # stride < nb
+    assert lib.fathom_nibbles_tm_from_planes(fake, 1, 128, 1000, 16, ctypes.c_void_p(264), n) == fathom.ERR_UNSUPPORTED
     ua = lib.fathom_union_attention
     assert ua(n, n, 0, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 0, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # M = 0
     assert ua(n, n, 2, 1, 64, 128, 64 * 128, 128, n, 4, n, n, 8, 1.0, n, n, 0, n) == fathom.ERR_INVALID_ARG   # dtype
